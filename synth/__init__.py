@@ -1,0 +1,172 @@
+"""Seeded synthetic inputs for the attention workloads.
+
+This module is shared by the CUDA path's tests and bench and by the float64
+oracle's callers. It draws random tensors and rounds them to the storage dtype.
+It holds none of the attention arithmetic.
+
+Recipe. Every (tensor, batch, head) slice has its own NumPy PCG64 stream seeded
+with SeedSequence([seed, tensor_id, b, h]). A slice can therefore be
+regenerated on its own, which lets the oracle rebuild only the heads it
+samples. Values are iid N(0, 1) float32, multiplied by `std`. For bf16
+workloads they are then rounded to the nearest bf16, ties to even, so the
+GPU and the oracle receive bit-identical numbers. The oracle upcasts them
+exactly to float64.
+
+Workloads (shapes from the pages' long-context regime; all synthetic, no dataset):
+  c1  fp32 fwd,  B=1 H=1 N=128 d=64, non-causal
+  c2  bf16 fwd+bwd, B=4 H=16 N=2048 d=64, causal, 1% of query rows x20
+  c3  bf16 fwd+bwd, B=2 H=32 N=8192 d=128, causal, std 1/sqrt(2)
+  c4  bf16 fwd,  B=1 H=16 N=65536 d=128, causal
+  c5  bf16 fwd+bwd GQA, B=1 Hq=32 Hkv=8 N=32768 d=128, causal
+"""
+from __future__ import annotations
+
+import concurrent.futures as _cf
+import math
+import os
+from dataclasses import dataclass, field
+
+import numpy as np
+
+# tensor ids used in the per-slice seed
+TID_Q, TID_K, TID_V, TID_DO, TID_SPIKE = 0, 1, 2, 3, 4
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    causal: bool
+    dtype: str  # "f32" or "bf16"
+    backward: bool
+    seed: int
+    std: float = 1.0
+    spike_frac: float = 0.0  # fraction of query rows per (b, h) multiplied by spike_mul
+    spike_mul: float = 1.0
+    # oracle sampling for the large shapes: (b, hq) heads and number of query rows
+    sample_heads: tuple = field(default=())
+    sample_rows: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+    def fwd_flops(self) -> float:
+        f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    def bwd_flops(self) -> float:
+        return 2.5 * self.fwd_flops()
+
+
+WORKLOADS = {
+    "c1": Workload("c1", 1, 1, 1, 128, 64, False, "f32", False, 1001),
+    "c2": Workload("c2", 4, 16, 16, 2048, 64, True, "bf16", True, 1002,
+                   spike_frac=0.01, spike_mul=20.0),
+    "c3": Workload("c3", 2, 32, 32, 8192, 128, True, "bf16", True, 1003,
+                   std=1.0 / math.sqrt(2.0),
+                   sample_heads=((0, 0), (0, 17), (1, 6), (1, 31)), sample_rows=256),
+    "c4": Workload("c4", 1, 16, 16, 65536, 128, True, "bf16", False, 1004,
+                   sample_heads=((0, 0), (0, 5), (0, 10), (0, 15)), sample_rows=256),
+    "c5": Workload("c5", 1, 32, 8, 32768, 128, True, "bf16", True, 1005,
+                   sample_heads=((0, 0), (0, 1), (0, 2), (0, 3),
+                                 (0, 28), (0, 29), (0, 30), (0, 31)), sample_rows=256),
+}
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bf16 (ties to even); returns float32."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32)
+    bias = ((u >> 16) & np.uint32(1)) + np.uint32(0x7FFF)
+    r = ((u + bias) & np.uint32(0xFFFF0000)).astype(np.uint32)
+    return r.view(np.float32)
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Upper 16 bits of float32 values that are already bf16-representable."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    return (x.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _rng(seed: int, tid: int, b: int, h: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, tid, b, h])))
+
+
+def head_slice(w: Workload, tid: int, b: int, h: int, n: int | None = None) -> np.ndarray:
+    """One [N, d] float32 slice of tensor `tid` for (b, h), already in storage precision."""
+    n = w.N if n is None else n
+    x = _rng(w.seed, tid, b, h).standard_normal((n, w.d), dtype=np.float32)
+    if w.std != 1.0:
+        x *= np.float32(w.std)
+    if tid == TID_Q and w.spike_frac > 0.0:
+        k = int(round(w.spike_frac * n))
+        rows = _rng(w.seed, TID_SPIKE, b, h).permutation(n)[:k]
+        x[rows] *= np.float32(w.spike_mul)
+    if w.dtype == "bf16":
+        x = round_to_bf16(x)
+    return x
+
+
+def spiked_rows(w: Workload, b: int, h: int) -> np.ndarray:
+    """The query rows of (b, h) that `head_slice` scaled by spike_mul."""
+    if w.spike_frac <= 0.0:
+        return np.zeros(0, dtype=np.int64)
+    k = int(round(w.spike_frac * w.N))
+    return np.sort(_rng(w.seed, TID_SPIKE, b, h).permutation(w.N)[:k])
+
+
+def _fill(args):
+    w, tid, b, h, out = args
+    out[b, h] = head_slice(w, tid, b, h)
+
+
+def tensor(w: Workload, tid: int, workers: int | None = None) -> np.ndarray:
+    """Full [B, H, N, d] float32 tensor (H = Hq for Q/dO, Hkv for K/V)."""
+    H = w.Hq if tid in (TID_Q, TID_DO) else w.Hkv
+    out = np.empty((w.B, H, w.N, w.d), dtype=np.float32)
+    jobs = [(w, tid, b, h, out) for b in range(w.B) for h in range(H)]
+    workers = workers or min(len(jobs), os.cpu_count() or 1)
+    if workers <= 1 or len(jobs) == 1:
+        for j in jobs:
+            _fill(j)
+    else:
+        with _cf.ThreadPoolExecutor(workers) as ex:
+            list(ex.map(_fill, jobs))
+    return out
+
+
+def small(B, Hq, Hkv, N, d, causal, seed, dtype="bf16", std=1.0, backward=True,
+          spike_frac=0.0, spike_mul=1.0) -> Workload:
+    """An ad-hoc workload for parity tests at small sizes."""
+    return Workload(f"t{B}x{Hq}x{Hkv}x{N}x{d}{'c' if causal else ''}", B, Hq, Hkv, N, d,
+                    causal, dtype, backward, seed, std=std, spike_frac=spike_frac,
+                    spike_mul=spike_mul)
+
+
+def sample_rows(w: Workload, b: int, h: int, count: int | None = None) -> np.ndarray:
+    """Sorted query (or key) row indices checked for a large workload.
+
+    Always includes the first rows, the tile edges at 127/128, the middle and the
+    last row, then seeded random rows up to `count`.
+    """
+    count = count or w.sample_rows or w.N
+    fixed = {0, 1, 127, 128, w.N // 2, w.N - 1}
+    fixed = {r for r in fixed if 0 <= r < w.N}
+    rng = _rng(w.seed, 99, b, h)
+    extra = rng.choice(w.N, size=min(w.N, count + len(fixed)), replace=False)
+    rows = list(sorted(fixed))
+    for r in extra:
+        if len(rows) >= count:
+            break
+        if r not in fixed:
+            rows.append(int(r))
+    return np.array(sorted(set(rows)), dtype=np.int64)
