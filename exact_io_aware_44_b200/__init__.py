@@ -1,0 +1,177 @@
+"""Exact IO-aware attention for NVIDIA B200 (sm_100a): Python binding.
+
+A thin ctypes layer over the C ABI in include/fa.h (libfa_b200.so, built
+in-tree by `python -m exact_io_aware_44_b200.build`). It only marshals
+arguments: it checks shapes and dtypes, allocates outputs with torch, and
+passes raw device pointers and the current CUDA stream. Every step of the
+attention path runs in the library's CUDA kernels. There is no CPU fallback:
+importing this package fails if the library is missing.
+
+    o, lse = fwd(q, k, v, causal=True)           # bf16 (tensor cores) or fp32
+    dq, dk, dv = bwd(q, k, v, o, lse, do, causal=True)
+
+Layouts: q, o, do: [B, Hq, N, d]; k, v: [B, Hkv, N, d]; lse: [B, Hq, N] float32.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = ["fwd", "bwd", "fwd_raw", "bwd_raw", "workspace_bytes", "get_status", "set_wait_budget_ns",
+           "selftest_wait_timeout", "FAError", "LIB_PATH", "lib", "STATUS"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
+
+STATUS = {0: "FA_OK", -1: "FA_ERR_INVALID_ARG", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_ALIGNMENT",
+          -4: "FA_ERR_LAUNCH", -5: "FA_ERR_DEVICE_TIMEOUT", -6: "FA_ERR_NO_DEVICE"}
+
+# exported symbols and their C signatures (must match include/fa.h)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+SIGNATURES = {
+    "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_get_status": (_I, [_P]),
+    "fa_set_wait_budget_ns": (None, [ctypes.c_uint64]),
+    "fa_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
+    "fa_error_string": (ctypes.c_char_p, [_I]),
+    "fa_version": (_I, []),
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        msg = lib.fa_error_string(code).decode() if lib is not None else STATUS.get(code, "?")
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({msg})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_44_b200.build` "
+                          "(there is no CPU fallback)")
+    so = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(so, name)
+        fn.restype = res
+        fn.argtypes = args
+    return so
+
+
+lib = _load()
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise FAError(code, where)
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dims(q, k):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, N, d]")
+    B, Hq, N, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, Nk, dk) != (B, N, d):
+        raise ValueError(f"k shape {tuple(k.shape)} does not match q shape {tuple(q.shape)}")
+    return B, Hq, Hkv, N, d
+
+
+def _require(t, name, dtype, device):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def fwd_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, N, d, causal, scale, stream_ptr, f32=False):
+    """The C call itself on raw device pointers (ints); returns the status code."""
+    fn = lib.fa_fwd_f32 if f32 else lib.fa_fwd
+    return fn(_P(q_ptr), _P(k_ptr), _P(v_ptr), _P(o_ptr), _P(lse_ptr), B, Hq, Hkv, N, d, int(bool(causal)),
+              float(scale), _P(stream_ptr))
+
+
+def fwd(q, k, v, causal: bool = True, scale: float | None = None, out=None, lse=None, stream=None):
+    """Forward pass. bf16 inputs run on the tensor cores (d in {64, 128});
+    float32 inputs run the fp32 CUDA-core kernel. Returns (o, lse)."""
+    import torch
+    B, Hq, Hkv, N, d = _dims(q, k)
+    dtype = q.dtype
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("q, k, v must be bfloat16 or float32")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n, dtype, q.device)
+    if v.shape != k.shape:
+        raise ValueError("v must have the shape of k")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _require(out, "out", dtype, q.device)
+    _require(lse, "lse", torch.float32, q.device)
+    fn = lib.fa_fwd_f32 if dtype == torch.float32 else lib.fa_fwd
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d, int(bool(causal)), scale,
+              _stream_ptr(stream)), "fa_fwd")
+    return out, lse
+
+
+def workspace_bytes(B, Hq, Hkv, N, d) -> int:
+    return int(lib.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d))
+
+
+def bwd_raw(q, k, v, o, lse, do, dq, dk, dv, ws, B, Hq, Hkv, N, d, causal, scale, stream_ptr):
+    """The C call itself on raw device pointers (ints); returns the status code."""
+    return lib.fa_bwd(_P(q), _P(k), _P(v), _P(o), _P(lse), _P(do), _P(dq), _P(dk), _P(dv), _P(ws), B, Hq, Hkv, N,
+                      d, int(bool(causal)), float(scale), _P(stream_ptr))
+
+
+def bwd(q, k, v, o, lse, do, causal: bool = True, scale: float | None = None, workspace=None, out=None,
+        stream=None):
+    """Backward pass (bf16). Returns (dq, dk, dv)."""
+    import torch
+    B, Hq, Hkv, N, d = _dims(q, k)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _require(t, n, torch.bfloat16, q.device)
+    _require(lse, "lse", torch.float32, q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    nbytes = workspace_bytes(B, Hq, Hkv, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    elif workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace needs {nbytes} bytes")
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    dq, dk, dv = out
+    _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                      _ptr(workspace), B, Hq, Hkv, N, d, int(bool(causal)), scale, _stream_ptr(stream)), "fa_bwd")
+    return dq, dk, dv
+
+
+def get_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(lib.fa_get_status(_stream_ptr(stream)))
+
+
+def set_wait_budget_ns(ns: int):
+    lib.fa_set_wait_budget_ns(int(ns))
+
+
+def selftest_wait_timeout(budget_ns: int = 10_000_000, stream=None) -> int:
+    return int(lib.fa_selftest_wait_timeout(int(budget_ns), _stream_ptr(stream)))

@@ -1,0 +1,277 @@
+// fa_api.cu -- the library's C ABI (declared in include/fa.h): argument
+// validation, TMA descriptor encoding, the device status word, and launches.
+// Nothing here computes attention; every step of the path runs in the kernels.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace fa {
+
+// First device-side error since the last fa_get_status(); 0 = none.
+__device__ int g_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<uint64_t> g_wait_budget_ns{2000000000ull};
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+struct DeviceInfo {
+  int checked = 0;  // 0 = not yet, 1 = sm_100, -1 = not sm_100
+  int* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Current device if it is an sm_100 part, with its status-word address.
+int current_device(DeviceInfo** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (di.checked == 0) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_NO_DEVICE;
+    }
+    if (major != 10) {
+      di.checked = -1;
+    } else {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+      }
+      di.status = static_cast<int*>(ptr);
+      di.checked = 1;
+    }
+  }
+  if (di.checked != 1) return FA_ERR_NO_DEVICE;
+  *out = &di;
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Common size checks. Returns FA_OK, or the code to return; *empty is set when
+// there is nothing to do.
+int check_sizes(int B, int Hq, int Hkv, int N, int d, float scale, bool* empty) {
+  *empty = false;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 0 || d < 1) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if ((long long)B * Hq * (long long)N >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  if (N == 0) *empty = true;
+  return FA_OK;
+}
+
+// 3-D bf16 tensor map over [heads, N, d] with a 64 x 128 box and the
+// 128-byte swizzle; rows past N read as zero.
+int make_map(CUtensorMap* m, const void* base, int d, int N, int heads) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc) return FA_ERR_LAUNCH;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kTileM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char* fa_error_string(int code) {
+  switch (code) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported shape";
+    case FA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case FA_ERR_LAUNCH: return "CUDA launch or query failed";
+    case FA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    case FA_ERR_NO_DEVICE: return "no sm_100 device is current";
+    default: return "unknown status";
+  }
+}
+
+void fa_set_wait_budget_ns(uint64_t ns) {
+  if (ns < 100000ull) ns = 100000ull;
+  if (ns > 60000000000ull) ns = 60000000000ull;
+  g_wait_budget_ns.store(ns);
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d,
+           int causal, float scale, void* stream) {
+  bool empty;
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
+  if (rc != FA_OK) return rc;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  DeviceInfo* di;
+  if ((rc = current_device(&di)) != FA_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_map(&tq, q, d, N, B * Hq)) != FA_OK) return rc;
+  if ((rc = make_map(&tk, k, d, N, B * Hkv)) != FA_OK) return rc;
+  if ((rc = make_map(&tv, v, d, N, B * Hkv)) != FA_OK) return rc;
+  FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.status = di->status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.causal = causal ? 1 : 0;
+  p.n_qblk = (N + 2 * kTileM - 1) / (2 * kTileM);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_budget_ns = g_wait_budget_ns.load();
+  if (launch_fwd_bf16(tq, tk, tv, p, d, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Hq, int Hkv, int N,
+               int d, int causal, float scale, void* stream) {
+  bool empty;
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
+  if (rc != FA_OK) return rc;
+  if (d % 4 != 0 || d > 128) return FA_ERR_UNSUPPORTED;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  DeviceInfo* di;
+  if ((rc = current_device(&di)) != FA_OK) return rc;
+  FwdF32Params p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.d = d;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (launch_fwd_f32(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
+  bool empty;
+  if (check_sizes(B, Hq, Hkv, N, d, 1.f, &empty) != FA_OK) return 0;
+  const size_t rows = (size_t)B * Hq * N;
+  const size_t delta = (rows * sizeof(float) + 255) & ~size_t(255);
+  return delta + rows * (size_t)d * sizeof(float);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+           void* dk, void* dv, void* workspace, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+           void* stream) {
+  bool empty;
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
+  if (rc != FA_OK) return rc;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_ALIGNMENT;
+  DeviceInfo* di;
+  if ((rc = current_device(&di)) != FA_OK) return rc;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((rc = make_map(&tq, q, d, N, B * Hq)) != FA_OK) return rc;
+  if ((rc = make_map(&tk, k, d, N, B * Hkv)) != FA_OK) return rc;
+  if ((rc = make_map(&tv, v, d, N, B * Hkv)) != FA_OK) return rc;
+  if ((rc = make_map(&tdo, dout, d, N, B * Hq)) != FA_OK) return rc;
+  const size_t rows = (size_t)B * Hq * N;
+  const size_t delta_bytes = (rows * sizeof(float) + 255) & ~size_t(255);
+  BwdParams p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.delta = static_cast<float*>(workspace);
+  p.dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + delta_bytes);
+  p.status = di->status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.d = d;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_budget_ns = g_wait_budget_ns.load();
+  if (launch_bwd_bf16(tq, tk, tv, tdo, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+int fa_get_status(void* stream) {
+  DeviceInfo* di;
+  int rc = current_device(&di);
+  if (rc != FA_OK) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  int v = 0;
+  if (cudaMemcpy(&v, di->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_LAUNCH;
+  const int zero = 0;
+  if (v != 0 && cudaMemcpy(di->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  return v;
+}
+
+int fa_selftest_wait_timeout(uint64_t budget_ns, void* stream) {
+  DeviceInfo* di;
+  int rc = current_device(&di);
+  if (rc != FA_OK) return rc;
+  if (budget_ns < 1000ull) budget_ns = 1000ull;
+  if (budget_ns > 2000000000ull) budget_ns = 2000000000ull;
+  if (launch_wait_selftest(di->status, budget_ns, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  return fa_get_status(stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,415 @@
+// fa_fwd_sm100.cu -- bf16 attention forward on sm_100a tensor cores.
+//
+// The method is the tiled forward with the online softmax: each query tile
+// streams the key/value tiles through on-chip memory, keeps a running row max m
+// and denominator l, rescales the partial output when m grows, and divides by l
+// once at the end ("FlashAttention Kernel & Online Softmax", first paragraph;
+// "FlashAttention" blog, mechanics of the running m, ell and O). The N x N score
+// matrix only ever exists as one 128 x 128 tile in Tensor Memory.
+//
+// One CTA owns two 128-row query tiles of one (batch, head) and 384 threads:
+//   warp 0      TMA producer: Q once, then K_j / V_j tiles through a ring of
+//               shared-memory stages guarded by mbarriers (full / empty).
+//   warp 1      allocates Tensor Memory; one lane issues every tcgen05.mma:
+//               S_t = Q_t K_j^T into TMEM, then O_t += P_t V_j into TMEM.
+//   warps 4-7   softmax for query tile 0 (thread = query row = TMEM lane).
+//   warps 8-11  softmax for query tile 1.
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 [384,384+d).
+//
+// Per key tile j, a softmax thread loads its row of S_t, applies the causal
+// mask on the diagonal tile, updates the running max, and computes
+// P = 2^(S c - m c) with c = scale * log2(e) on the SFU. It rescales its row
+// of O_t in TMEM only when the max grew by more than 2^8; otherwise the stale
+// max stays the reference, which is exact because the final division uses the
+// same reference. P is written to shared memory as bf16 in the 128-byte-swizzled
+// K-major layout that tcgen05.mma reads. The epilogue divides O by l, stores O
+// as bf16 and writes LSE = (m c + log2 l) ln 2.
+//
+// The MMA issue order per key tile j is S_0(j), S_1(j), PV_0(j-1), PV_1(j-1),
+// so the tensor core computes the next scores while both softmax warpgroups
+// exponentiate the current ones. The shared-memory ring holds tiles in the
+// same order: K_0, K_1, V_0, K_2, V_1, ..., V_last.
+#include <math.h>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kFwdThreads = 384;
+// Register split: 384 threads x 168 at launch = 64512 = 128 x 56 (producer /
+// MMA warpgroup) + 256 x 224 (the two softmax warpgroups).
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsControl = 56;
+constexpr int kRegsSoftmax = 224;
+static_assert(kFwdThreads * kRegsLaunch == 128 * kRegsControl + 256 * kRegsSoftmax, "register split");
+constexpr uint32_t kRescaleThresholdLog2 = 8;  // rescale only when m grows by > 2^8
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kStages = (D == 128) ? 3 : 6;
+  static constexpr int kTileBytes = kTileM * D * 2;      // one Q, K or V tile (bf16)
+  static constexpr int kPBytes = kTileM * kTileN * 2;    // one P tile (bf16)
+  static constexpr int kRegion = kTileM * 128;           // one 64-column block of a tile
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffP = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffKV = kOffP + 2 * kPBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  // q_full, ring_full[S], ring_empty[S], s_ready[2], s_free[2], p_ready[2], pv_done[2], mma_final
+  static constexpr int kNumBars = 1 + 2 * kStages + 9;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* ring_full = bars + 1;
+  uint64_t* ring_empty = ring_full + S;
+  uint64_t* s_ready = ring_empty + S;
+  uint64_t* s_free = s_ready + 2;
+  uint64_t* p_ready = s_free + 2;
+  uint64_t* pv_done = p_ready + 2;
+  uint64_t* mma_final = pv_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Work unit: head-major so that concurrently running CTAs share K/V in L2,
+  // and within a head the longest (last) query blocks first.
+  const int bh = blockIdx.x / p.n_qblk;
+  const int qb = p.n_qblk - 1 - (blockIdx.x % p.n_qblk);
+  const int b = bh / p.Hq;
+  const int h = bh % p.Hq;
+  const int kv_head = b * p.Hkv + h / (p.Hq / p.Hkv);
+  const int q0 = qb * 2 * kTileM;
+  const int n_kv_all = (p.N + kTileN - 1) / kTileN;
+  int n_iter[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = q0 / kTileM + t;  // index of this query tile
+    const bool active = q0 + t * kTileM < p.N;
+    n_iter[t] = !active ? 0 : (p.causal ? qt + 1 : n_kv_all);
+  }
+  const int n_kv = max(n_iter[0], n_iter[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&ring_full[s], 1);
+      mbar_init(&ring_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_ready[t], 1);
+      mbar_init(&s_free[t], kTileM);
+      mbar_init(&p_ready[t], kTileM);
+      mbar_init(&pv_done[t], 1);
+    }
+    mbar_init(mma_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx w{abort_flag, p.status, p.wait_budget_ns};
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    regs_dec<kRegsControl>();
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const int q_head = b * p.Hq + h;
+      const int n_qt = n_iter[1] > 0 ? 2 : 1;
+      mbar_arrive_expect_tx(q_full, n_qt * C::kTileBytes);
+      for (int t = 0; t < n_qt; ++t)
+#pragma unroll
+        for (int z = 0; z < D / 64; ++z)
+          tma_load_3d(smem + C::kOffQ + t * C::kTileBytes + z * C::kRegion, &tmQ, q_full, z * 64,
+                      q0 + t * kTileM, q_head);
+      int it = 0;
+      auto push = [&](const CUtensorMap* map, int kv_tile) -> bool {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
+        if (!mbar_wait(&ring_empty[s], ph ^ 1, w)) return false;
+        mbar_arrive_expect_tx(&ring_full[s], C::kTileBytes);
+#pragma unroll
+        for (int z = 0; z < D / 64; ++z)
+          tma_load_3d(smem + C::kOffKV + s * C::kTileBytes + z * C::kRegion, map, &ring_full[s], z * 64,
+                      kv_tile * kTileN, kv_head);
+        ++it;
+        return true;
+      };
+      bool ok = true;
+      for (int j = 0; j < n_kv && ok; ++j) {
+        ok = push(&tmK, j);
+        if (ok && j >= 1) ok = push(&tmV, j - 1);
+      }
+      if (ok) ok = push(&tmV, n_kv - 1);
+      if (!ok) {
+        // Error path: let the loads already issued land before the CTA exits.
+        WaitCtx drain{abort_flag, p.status, 20000000ull};
+        volatile int zero = 0;
+        drain.abort_flag = &zero;
+        for (int k = max(0, it - S); k < it; ++k) mbar_wait(&ring_full[k % S], (k / S) & 1, drain);
+        mbar_wait(q_full, 0, drain);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    regs_dec<kRegsControl>();
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
+      constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, false, true);
+      const uint32_t q_base = smem_u32(smem + C::kOffQ);
+      const uint32_t p_base = smem_u32(smem + C::kOffP);
+      const uint32_t kv_base = smem_u32(smem + C::kOffKV);
+      int it = 0;
+      bool ok = mbar_wait(q_full, 0, w);
+      tc_fence_after();
+      auto take = [&](int& slot) -> bool {
+        slot = it % S;
+        const bool r = mbar_wait(&ring_full[slot], (it / S) & 1, w);
+        ++it;
+        tc_fence_after();
+        return r;
+      };
+      auto issue_s = [&](int t, int slot) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * C::kRegion + (k & 3) * 32;
+          const uint64_t a = sdesc_sw128(q_base + t * C::kTileBytes + off, 16, 1024);
+          const uint64_t bd = sdesc_sw128(kv_base + slot * C::kTileBytes + off, 16, 1024);
+          mma_bf16_ss(tmem + t * 128, a, bd, kIdescS, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_ready[t]);
+      };
+      auto issue_pv = [&](int t, int slot, int j) {
+#pragma unroll
+        for (int k = 0; k < kTileN / 16; ++k) {
+          const uint64_t a = sdesc_sw128(p_base + t * C::kPBytes + (k >> 2) * C::kRegion + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(kv_base + slot * C::kTileBytes + k * 16 * 128, C::kRegion, 1024);
+          mma_bf16_ss(tmem + 256 + t * 128, a, bd, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&pv_done[t]);
+      };
+      auto do_pv = [&](int j) -> bool {  // PV_0(j), PV_1(j) from the V_j stage
+        int slot;
+        if (!take(slot)) return false;
+        for (int t = 0; t < 2; ++t) {
+          if (j >= n_iter[t]) continue;
+          if (!mbar_wait(&p_ready[t], j & 1, w)) return false;
+          tc_fence_after();
+          issue_pv(t, slot, j);
+        }
+        mma_commit(&ring_empty[slot]);
+        return true;
+      };
+      for (int j = 0; j < n_kv && ok; ++j) {
+        int slot;
+        ok = take(slot);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= n_iter[t]) continue;
+          if (j > 0) {
+            ok = mbar_wait(&s_free[t], (j - 1) & 1, w);
+            tc_fence_after();
+          }
+          if (ok) issue_s(t, slot);
+        }
+        if (!ok) break;
+        mma_commit(&ring_empty[slot]);
+        if (j >= 1) ok = do_pv(j - 1);
+      }
+      if (ok) ok = do_pv(n_kv - 1);
+      // Every MMA issued above must finish before TMEM is released.
+      mma_commit(mma_final);
+      WaitCtx drain{abort_flag, p.status, 20000000ull};
+      volatile int zero = 0;
+      drain.abort_flag = &zero;
+      mbar_wait(mma_final, 0, drain);
+    }
+  } else if (warp < 4) {
+    regs_dec<kRegsControl>();
+  } else {
+    // ------------------------------------------------------------ softmax
+    regs_inc<kRegsSoftmax>();
+    const int t = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int n = n_iter[t];
+    if (n > 0) {
+      const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+      const uint32_t tS = tmem + lane_off + t * 128;
+      const uint32_t tO = tmem + lane_off + 256 + t * 128;
+      const uint32_t p_tile = smem_u32(smem + C::kOffP + t * C::kPBytes);
+      const int qrow = q0 + t * kTileM + row;
+      const float c = p.scale_log2;
+      float m_ref = -INFINITY;  // reference max (raw score units)
+      float l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n; ++j) {
+        if (!(ok = mbar_wait(&s_ready[t], j & 1, w))) break;
+        tc_fence_after();
+        float s[kTileN];
+#pragma unroll
+        for (int cc = 0; cc < kTileN / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(tS + cc * 32, r);
+          tmem_ld_wait(r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
+        }
+        tc_fence_before();
+        mbar_arrive(&s_free[t]);
+
+        const int k0 = j * kTileN;
+        if (p.causal && j == n - 1) {
+          const int lim = qrow - k0;  // keys with column > lim are in the future
+#pragma unroll
+          for (int i = 0; i < kTileN; ++i)
+            if (i > lim) s[i] = -INFINITY;
+        } else if (!p.causal && j == n - 1 && p.N - k0 < kTileN) {
+          const int lim = p.N - k0;
+#pragma unroll
+          for (int i = 0; i < kTileN; ++i)
+            if (i >= lim) s[i] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int i = 1; i < kTileN; ++i) mx = fmaxf(mx, s[i]);
+        const float m_new = fmaxf(m_ref, mx);
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m_ref = m_new;
+        } else if ((m_new - m_ref) * c > (float)kRescaleThresholdLog2) {
+          alpha = ex2((m_ref - m_new) * c);
+          m_ref = m_new;
+          l *= alpha;
+          rescale = true;
+        }
+        const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+        // P = 2^(S c - m c), packed to bf16 pairs at once; l sums the fp32 values.
+        uint32_t pk[kTileN / 2];
+        float rs = 0.f;
+#pragma unroll
+        for (int i = 0; i < kTileN; i += 2) {
+          const float e0 = ex2(fmaf(s[i], c, -mc));
+          const float e1 = ex2(fmaf(s[i + 1], c, -mc));
+          rs += e0 + e1;
+          pk[i / 2] = pack_bf16x2(e0, e1);
+        }
+        l += rs;
+
+        if (j >= 1) {
+          // PV(j-1) must be done: it reads the P buffer and accumulates into O.
+          if (!(ok = mbar_wait(&pv_done[t], (j - 1) & 1, w))) break;
+          tc_fence_after();
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld32(tO + cc * 32, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(tO + cc * 32, r);
+          }
+          tmem_st_wait();
+        }
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const int c2 = (z * 64 + ch * 8) / 2;
+            st_shared_v4(p_tile + z * C::kRegion + sw128_offset(row, ch), pk[c2], pk[c2 + 1], pk[c2 + 2],
+                         pk[c2 + 3]);
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&p_ready[t]);
+      }
+      if (ok && (ok = mbar_wait(&pv_done[t], (n - 1) & 1, w))) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        const bool valid = qrow < p.N;
+        const size_t row_idx = (size_t)(b * p.Hq + h) * p.N + qrow;
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row_idx * D);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(tO + cc * 32, r);
+          tmem_ld_wait(r);
+          if (valid) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              uint4 u;
+              const int i = v4 * 8;
+              u.x = pack_bf16x2(__uint_as_float(r[i + 0]) * inv_l, __uint_as_float(r[i + 1]) * inv_l);
+              u.y = pack_bf16x2(__uint_as_float(r[i + 2]) * inv_l, __uint_as_float(r[i + 3]) * inv_l);
+              u.z = pack_bf16x2(__uint_as_float(r[i + 4]) * inv_l, __uint_as_float(r[i + 5]) * inv_l);
+              u.w = pack_bf16x2(__uint_as_float(r[i + 6]) * inv_l, __uint_as_float(r[i + 7]) * inv_l);
+              dst[cc * 4 + v4] = u;
+            }
+          }
+        }
+        if (valid) p.lse[row_idx] = (m_ref * c + log2f(l)) * 0.6931471805599453f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                         cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const long long grid = (long long)p.B * p.Hq * p.n_qblk;
+  fwd_bf16_kernel<D><<<(unsigned)grid, kFwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, int d, cudaStream_t s) {
+  return d == 128 ? launch_fwd_d<128>(tq, tk, tv, p, s) : launch_fwd_d<64>(tq, tk, tv, p, s);
+}
+
+}  // namespace fa

@@ -1,0 +1,56 @@
+// fa_internal.h -- parameter blocks and launchers shared by the host C ABI
+// (fa_api.cu) and the kernel translation units. Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+constexpr int kTileM = 128;  // query rows per tile (TMEM lanes)
+constexpr int kTileN = 128;  // keys per tile
+
+struct FwdParams {
+  void* o;            // bf16 [B, Hq, N, d]
+  float* lse;         // [B, Hq, N]
+  int* status;        // device status word
+  int B, Hq, Hkv, N;
+  int causal;
+  int n_qblk;         // query blocks of 2 tiles (256 rows) per head
+  float scale_log2;   // scale * log2(e)
+  uint64_t wait_budget_ns;
+};
+
+struct FwdF32Params {
+  const float *q, *k, *v;
+  float* o;
+  float* lse;
+  int B, Hq, Hkv, N, d;
+  int causal;
+  float scale_log2;
+};
+
+struct BwdParams {
+  const void *q, *k, *v, *o, *dout;
+  const float* lse;
+  void *dq, *dk, *dv;
+  float* delta;      // workspace: D = rowsum(dO o O), [B, Hq, N]
+  float* dq_acc;     // workspace: fp32 dQ accumulator, [B, Hq, N, d]
+  int* status;
+  int B, Hq, Hkv, N, d;
+  int causal;
+  float scale;
+  float scale_log2;
+  uint64_t wait_budget_ns;
+};
+
+// Launchers (return a cudaError_t from the launch).
+cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, int d, cudaStream_t s);
+cudaError_t launch_fwd_f32(const FwdF32Params& p, cudaStream_t s);
+cudaError_t launch_bwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const BwdParams& p, cudaStream_t s);
+cudaError_t launch_wait_selftest(int* status, uint64_t budget_ns, cudaStream_t s);
+
+}  // namespace fa

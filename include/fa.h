@@ -1,0 +1,150 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact IO-aware attention library.
+ *
+ * What the library computes. Exact scaled-dot-product attention
+ *     O = softmax(scale * Q K^T) V
+ * ("Walk through what FlashAttention does differently from standard attention",
+ * zenaique short answer, first paragraph: the textbook formula with scale 1/sqrt(d_k);
+ * FlashAttention returns the same output, only floating-point rounding differs).
+ * The score matrix is produced tile by tile in on-chip memory and merged with the
+ * online softmax (running max m, running denominator l, rescaled output accumulator;
+ * "FlashAttention Kernel & Online Softmax" card, first paragraph, and the
+ * "FlashAttention" blog's mechanics section). It never reaches device memory.
+ * The forward pass also saves each row's log-sum-exp (LSE), which folds the
+ * saved statistics m and l into one number. The backward pass recomputes the
+ * scores and probabilities from Q, K and that LSE instead of storing them (same
+ * short answer, second paragraph).
+ *
+ * Conventions shared by every entry point.
+ *   Layout    Q, O, dO, dQ: [B, Hq, N, d]; K, V, dK, dV: [B, Hkv, N, d]; all
+ *             contiguous, row-major, d innermost. LSE and the backward's D: [B, Hq, N].
+ *   Types     "bf16" arguments point to IEEE bfloat16 values (2 bytes each);
+ *             LSE is float32, natural logarithm.
+ *   Heads     Grouped-query attention: query head h reads key/value head
+ *             h / (Hq / Hkv). Hq must be a multiple of Hkv.
+ *   Causal    causal != 0: query i sees keys j <= i (square N x N). Otherwise all keys.
+ *   Scale     scale > 0 and finite, applied to Q K^T (callers normally pass 1/sqrt(d)).
+ *   Memory    Every pointer is DEVICE memory owned by the caller. Each pointer
+ *             must be 16-byte aligned. Outputs must not alias inputs.
+ *   Streams   `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *             asynchronous: they enqueue work and return before it completes.
+ *   Errors    A negative return code means nothing was launched and no output
+ *             was touched. FA_OK means the work was enqueued. A failure found on
+ *             the device is recorded in a device status word; fa_get_status()
+ *             reads it. On the device, every wait is bounded. A wait that runs
+ *             out records FA_ERR_DEVICE_TIMEOUT and the kernel returns early; it
+ *             never traps or spins forever.
+ *   Sizes     B, Hq, Hkv >= 1; N >= 0 (N == 0 is a no-op that returns FA_OK);
+ *             B*Hq*N < 2^31.
+ */
+#ifndef FA_B200_H_
+#define FA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = -1,    /* a size, scale or pointer argument is invalid        */
+  FA_ERR_UNSUPPORTED = -2,    /* valid, but not a supported shape (e.g. d not 64/128) */
+  FA_ERR_ALIGNMENT = -3,      /* a pointer is not 16-byte aligned                     */
+  FA_ERR_LAUNCH = -4,         /* the CUDA runtime refused a launch or a query         */
+  FA_ERR_DEVICE_TIMEOUT = -5, /* a bounded device-side wait ran out                   */
+  FA_ERR_NO_DEVICE = -6       /* no sm_100 device is current                          */
+} fa_status_t;
+
+/*
+ * fa_fwd -- bf16 forward pass on the tensor cores.
+ *
+ * Computes O = softmax(scale * Q K^T) V tile by tile with the online softmax
+ * ("FlashAttention Kernel & Online Softmax": m_new = max(m, x),
+ * l_new = l e^(m - m_new) + e^(x - m_new), output rescaled by e^(m - m_new) and
+ * normalised by 1/l at the end). It also writes lse[i] = m_i + ln(l_i) for
+ * every row (the statistics that the short answer's second paragraph says
+ * are saved for the backward pass).
+ *   q [B,Hq,N,d] bf16, k/v [B,Hkv,N,d] bf16   inputs (read only)
+ *   o [B,Hq,N,d] bf16                          output, round-to-nearest-even
+ *   lse [B,Hq,N] float32                       output
+ *   d must be 64 or 128. Arithmetic: bf16 operands, fp32 accumulation; the
+ *   probabilities P are rounded to bf16 before the P V product.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * fa_fwd_f32 -- float32 forward pass (CUDA cores, fp32 throughout).
+ *
+ * The same computation as fa_fwd, on float32 q, k, v and o. Tiles of queries
+ * and keys are staged in shared memory and merged with the same online
+ * softmax. d must be a multiple of 4 and at most 128.
+ */
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+               int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * fa_bwd_workspace_bytes -- device scratch that fa_bwd needs.
+ *
+ * The workspace holds D = rowsum(dO o O) (float32 [B,Hq,N]) and a float32
+ * accumulator for dQ ([B,Hq,N,d]). It grows linearly in N: the backward pass
+ * never stores an N x N matrix. Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * fa_bwd -- bf16 backward pass by recomputation.
+ *
+ * Gradients of L = sum(O o dO) with respect to Q, K and V. The backward pass
+ * recomputes S = scale Q K^T and P = exp(S - LSE) tile by tile from the saved
+ * LSE instead of storing them (short answer, second paragraph). With
+ * D_i = sum_c dO_ic O_ic and dS = P o (dP - D), where dP = dO V^T:
+ *   dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+ * With grouped-query attention, dK and dV sum over the query heads of a group.
+ *   q, k, v, o, dout  bf16 inputs (o and lse as written by fa_fwd)
+ *   lse               float32 [B,Hq,N] input
+ *   dq [B,Hq,N,d], dk, dv [B,Hkv,N,d]  bf16 outputs
+ *   workspace         at least fa_bwd_workspace_bytes(...) bytes of device
+ *                     memory, 256-byte aligned; its contents on entry do not matter.
+ *                     It must not be used by another call in flight at the same time.
+ *   d must be 64 or 128. dQ is accumulated with float32 atomics, so its last
+ *   bits can vary from run to run; dK and dV are deterministic.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, void* workspace,
+           int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * fa_get_status -- synchronise `stream`, then return and clear the device
+ * status word of the current device (FA_OK or the first device-side error
+ * since the last call). Returns FA_ERR_LAUNCH if the stream reports a CUDA error.
+ */
+int fa_get_status(void* stream);
+
+/* fa_set_wait_budget_ns -- budget of each bounded device-side wait (default
+ * 2e9 ns). Kernels launched afterwards use the new value. Values outside
+ * [1e5, 6e10] ns are clamped to that range. */
+void fa_set_wait_budget_ns(uint64_t ns);
+
+/*
+ * fa_selftest_wait_timeout -- failure-detection self test. Launches one block
+ * that waits on a shared-memory barrier that nothing ever completes, using a
+ * budget of `budget_ns`. The bounded wait must run out, record
+ * FA_ERR_DEVICE_TIMEOUT and return. The call synchronises `stream` and returns
+ * the status it read (FA_ERR_DEVICE_TIMEOUT when the mechanism works). It
+ * also clears the status word.
+ */
+int fa_selftest_wait_timeout(uint64_t budget_ns, void* stream);
+
+/* fa_error_string -- static text for a status code (never NULL). */
+const char* fa_error_string(int code);
+
+/* fa_version -- library version as 10000*major + 100*minor + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FA_B200_H_ */

@@ -19,3 +19,16 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(autouse=True, scope="session")
+def _short_device_waits():
+    """Device-side waits in tests give up after 1 s instead of the default 2 s."""
+    try:
+        import torch
+        if torch.cuda.is_available():
+            import exact_io_aware_44_b200 as fa
+            fa.set_wait_budget_ns(1_000_000_000)
+    except ImportError:
+        pass
+    yield

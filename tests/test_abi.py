@@ -1,0 +1,93 @@
+"""The C ABI boundary, checked without a GPU: the library loads, exports every
+symbol include/fa.h declares, and rejects invalid arguments on the host before
+any CUDA call (so nothing is launched and no output is touched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_io_aware_44_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "fa.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for s in ("fa_fwd", "fa_fwd_f32", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_status", "fa_error_string"):
+        assert s in syms
+
+
+def test_every_declared_symbol_is_exported():
+    so = ctypes.CDLL(fa.LIB_PATH)
+    for s in declared_symbols():
+        assert hasattr(so, s), s
+        assert s in fa.SIGNATURES, f"binding lacks {s}"
+
+
+def test_library_has_sm100a_code_only_and_static_runtime():
+    # the shared object must not need libcudart.so at load time
+    import subprocess
+    out = subprocess.run(["ldd", fa.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcudart.so" not in out
+    assert "libcuda.so" not in out
+
+
+def test_version_and_error_strings():
+    assert fa.lib.fa_version() >= 100
+    for code in list(fa.STATUS) + [12345]:
+        assert fa.lib.fa_error_string(code)
+
+
+def _fwd(d=64, B=1, Hq=2, Hkv=1, N=128, causal=1, scale=0.125, ptr=0x1000, f32=False):
+    return fa.fwd_raw(ptr, ptr, ptr, ptr, ptr, B, Hq, Hkv, N, d, causal, scale, 0, f32=f32)
+
+
+def test_invalid_arguments_rejected_on_host():
+    assert _fwd(d=96) == -2                       # unsupported head dim
+    assert _fwd(d=64, Hq=3, Hkv=2) == -1          # Hq not a multiple of Hkv
+    assert _fwd(B=0) == -1
+    assert _fwd(scale=0.0) == -1
+    assert _fwd(scale=float("nan")) == -1
+    assert _fwd(scale=float("inf")) == -1
+    assert _fwd(N=-1) == -1
+    assert _fwd(ptr=0x1008) == -3                 # not 16-byte aligned
+    assert _fwd(ptr=0) == -1                      # null pointers
+    assert _fwd(N=0, ptr=0) == 0                  # empty problem: nothing to do
+    assert _fwd(d=102, f32=True) == -2            # fp32 path: d % 4 != 0
+    assert _fwd(d=132, f32=True) == -2            # fp32 path: d > 128
+    assert _fwd(B=1 << 12, Hq=1 << 10, Hkv=1, N=1 << 10) == -2   # B*Hq*N >= 2^31
+
+
+def test_bwd_rejects_bad_arguments_on_host():
+    p = 0x1000
+    r = fa.bwd_raw(p, p, p, p, p, p, p, p, p, p + 16, 1, 2, 1, 128, 64, 1, 0.125, 0)
+    assert r == -3                                # workspace must be 256-byte aligned
+    r = fa.bwd_raw(p, p, p, p, p, p, p, p, p, 0, 1, 2, 1, 128, 64, 1, 0.125, 0)
+    assert r == -1
+    r = fa.bwd_raw(p, p, p, p, p, p, p, p, p, p, 1, 2, 1, 128, 80, 1, 0.125, 0)
+    assert r == -2
+
+
+def test_workspace_is_linear_in_n():
+    """The backward's scratch is O(N): D (fp32 per row) and the fp32 dQ accumulator."""
+    B, Hq, Hkv, d = 2, 8, 2, 128
+    sizes = [fa.workspace_bytes(B, Hq, Hkv, N, d) for N in (1024, 2048, 4096, 8192)]
+    per_row = B * Hq * (d + 1) * 4
+    for N, s in zip((1024, 2048, 4096, 8192), sizes):
+        assert per_row * N <= s <= per_row * N + 256
+    assert fa.workspace_bytes(0, 1, 1, 8, 64) == 0
+
+
+def test_no_device_is_reported_without_gpu():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _fwd() == -6
+    assert fa.lib.fa_get_status(None) == -6
