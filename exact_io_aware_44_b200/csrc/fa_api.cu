@@ -89,14 +89,14 @@ int check_sizes(int B, int Hq, int Hkv, int N, int d, float scale, bool* empty) 
   return FA_OK;
 }
 
-// 3-D bf16 tensor map over [heads, N, d] with a 64 x 128 box and the
-// 128-byte swizzle; rows past N read as zero.
-int make_map(CUtensorMap* m, const void* base, int d, int N, int heads) {
+// 3-D bf16 tensor map over [heads, N, d] with a 64-column x `box_rows` box and
+// the 128-byte swizzle; rows past N read as zero.
+int make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box_rows = kTileM) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return FA_ERR_LAUNCH;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)heads};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)kTileM, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -215,10 +215,11 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   DeviceInfo* di;
   if ((rc = current_device(&di)) != FA_OK) return rc;
   CUtensorMap tq, tk, tv, tdo;
-  if ((rc = make_map(&tq, q, d, N, B * Hq)) != FA_OK) return rc;
+  const int q_rows = (d == 128) ? 64 : 128;  // query rows per backward tile
+  if ((rc = make_map(&tq, q, d, N, B * Hq, q_rows)) != FA_OK) return rc;
   if ((rc = make_map(&tk, k, d, N, B * Hkv)) != FA_OK) return rc;
   if ((rc = make_map(&tv, v, d, N, B * Hkv)) != FA_OK) return rc;
-  if ((rc = make_map(&tdo, dout, d, N, B * Hq)) != FA_OK) return rc;
+  if ((rc = make_map(&tdo, dout, d, N, B * Hq, q_rows)) != FA_OK) return rc;
   const size_t rows = (size_t)B * Hq * N;
   const size_t delta_bytes = (rows * sizeof(float) + 255) & ~size_t(255);
   BwdParams p;

@@ -1,9 +1,580 @@
-// fa_bwd_sm100.cu -- placeholder until the backward kernels land.
+// fa_bwd_sm100.cu -- bf16 attention backward on sm_100a, by recomputation.
+//
+// The backward pass does not store the score matrix: it recomputes S and P
+// block by block from Q, K and the saved log-sum-exp ("Walk through what
+// FlashAttention does differently from standard attention", second paragraph:
+// the backward recomputes attention from the saved Q, K, V and statistics).
+// For L = sum(O o dO), with D_i = sum_c dO_ic O_ic and dS = P o (dP - D):
+//   dV = P^T dO,   dP = dO V^T,   dK = scale dS^T Q,   dQ = scale dS K.
+//
+// Three kernels:
+//   bwd_preprocess  D = rowsum(dO o O) (fp32) and zeroes the fp32 dQ accumulator.
+//   bwd_main        one CTA per 128-key tile of one (batch, kv head). It keeps K
+//                   and V in shared memory and dK, dV in Tensor Memory, and loops
+//                   over the query heads of its GQA group and the query tiles
+//                   that can see its keys. Per query tile i (BR rows):
+//                     S^T = K Q_i^T, dP^T = V dO_i^T          (tcgen05.mma -> TMEM)
+//                     P^T = 2^(S^T c - LSE_i log2 e), dS^T = P^T o (dP^T - D_i)
+//                     dV += P^T dO_i, dK += dS^T Q_i            (TMEM accumulators)
+//                     dQ_i partial = dS K (d = 64) or K^T dS^T (d = 128) -> TMEM,
+//                     then added to the fp32 accumulator with red.global.add.
+//   bwd_convert     dQ = bf16(scale * accumulator).
+//
+// bwd_main roles (384 threads):
+//   warp 0      producer: K, V once (TMA); per query tile Q_i, dO_i (TMA) and
+//               LSE_i log2(e), D_i (plain loads) into a ring of stages.
+//   warp 1      allocates TMEM; one lane issues every tcgen05.mma.
+//   warps 4-7   thread = key row: P^T and dS^T, written to shared memory in the
+//               128-byte-swizzled K-major layout.
+//   warps 8-11  thread = TMEM lane of the dQ tile: reads it and issues the fp32
+//               reductions; at the end, writes dK and dV.
+//
+// Query tiles are BR = 64 rows for d = 128 (so dQ^T = K^T dS^T has M = d = 128)
+// and BR = 128 rows for d = 64 (so dQ = dS K has M = 128 query rows). TMEM
+// columns: S^T [0, BR), dP^T [BR, 2BR), dQ [2BR, 2BR + 64), dV [512 - 2d, 512 - d),
+// dK [512 - d, 512).
+#include <math.h>
+
+#include <algorithm>
+
 #include "fa_internal.h"
+#include "sm100.cuh"
 
 namespace fa {
-cudaError_t launch_bwd_bf16(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                            const BwdParams&, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int kBwdThreads = 384;
+// Register split: the launch gives 168 per thread (384 x 168 = 64512). The
+// control warpgroup lowers to 56, the P/dS warpgroup raises to 232, and the dQ
+// warpgroup keeps the launch count: 128 x (56 + 232 + 168) = 58368 <= 64512.
+constexpr int kBwdRegsLaunch = 168;
+constexpr int kBwdRegsControl = 56;
+constexpr int kBwdRegsSoftmax = 232;
+static_assert(128 * (kBwdRegsControl + kBwdRegsSoftmax + kBwdRegsLaunch) <= kBwdThreads * kBwdRegsLaunch,
+              "register split");
+
+template <int D>
+struct BwdCfg {
+  static constexpr int BR = (D == 128) ? 64 : 128;  // query rows per tile
+  static constexpr int kStages = 3;
+  static constexpr int kKVBytes = kTileN * D * 2;   // K or V tile (128 keys)
+  static constexpr int kKVRegion = kTileN * 128;    // 64-column block of a K/V tile
+  static constexpr int kQBytes = BR * D * 2;        // Q or dO tile
+  static constexpr int kQRegion = BR * 128;         // 64-column block of a Q/dO tile
+  static constexpr int kPBytes = kTileN * BR * 2;   // P^T or dS^T tile (128 keys x BR queries)
+  static constexpr int kPRegion = kTileN * 128;
+  static constexpr int kStageBytes = 2 * kQBytes + 1024;  // Q, dO, then LSE2 and D vectors
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kKVBytes;
+  static constexpr int kOffStage = kOffV + kKVBytes;
+  static constexpr int kOffP = kOffStage + kStages * kStageBytes;
+  static constexpr int kOffDS = kOffP + kPBytes;
+  static constexpr int kOffBar = kOffDS + kPBytes;
+  // kv_full, st_full[S], st_empty[S], s_full, s_free, dp_full, dp_free, p_full, p_free,
+  // ds_full, ds_free, dq_full, dq_free, mma_done
+  static constexpr int kNumBars = 1 + 2 * kStages + 11;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  // TMEM columns
+  static constexpr int kColS = 0;
+  static constexpr int kColDP = BR;
+  static constexpr int kColDQ = 2 * BR;
+  static constexpr int kColDV = 512 - 2 * D;
+  static constexpr int kColDK = 512 - D;
+  static_assert(kColDQ + 64 <= kColDV, "TMEM layout");
+};
+
+__device__ __forceinline__ uint8_t* align1024b(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+__device__ __forceinline__ void red_add(float* p, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// D = rowsum(dO o O); dQ accumulator = 0. One thread per 8 columns of a row.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
+                                                             const __nv_bfloat16* __restrict__ dout,
+                                                             float* __restrict__ delta, float* __restrict__ dq_acc,
+                                                             long long rows) {
+  constexpr int kPer = D / 8;  // threads per row (16 or 8)
+  const long long total = rows * kPer;
+  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t - threadIdx.x < total;
+       t += (long long)gridDim.x * blockDim.x) {
+    const bool in = t < total;
+    const long long row = t / kPer;
+    const int part = (int)(t % kPer);
+    float acc = 0.f;
+    if (in) {
+      const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
+      const uint4 b = *reinterpret_cast<const uint4*>(dout + row * D + part * 8);
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(a2[i]);
+        const float2 y = __bfloat1622float2(b2[i]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+      float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int off = kPer / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (in && part == 0) delta[row] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ = bf16(scale * accumulator), 8 elements per thread.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) bwd_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
+                                                          long long n8, float scale) {
+  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n8; t += (long long)gridDim.x * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * t];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * t + 1];
+    uint4 u;
+    u.x = pack_bf16x2(a.x * scale, a.y * scale);
+    u.y = pack_bf16x2(a.z * scale, a.w * scale);
+    u.z = pack_bf16x2(b.x * scale, b.y * scale);
+    u.w = pack_bf16x2(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dq)[t] = u;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// main backward kernel
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int BR = C::BR;
+  constexpr int ST = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024b(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_full = bars;
+  uint64_t* st_full = bars + 1;
+  uint64_t* st_empty = st_full + ST;
+  uint64_t* s_full = st_empty + ST;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* dp_full = s_free + 1;
+  uint64_t* dp_free = dp_full + 1;
+  uint64_t* p_full = dp_free + 1;
+  uint64_t* p_free = p_full + 1;
+  uint64_t* ds_full = p_free + 1;
+  uint64_t* ds_free = ds_full + 1;
+  uint64_t* dq_full = ds_free + 1;
+  uint64_t* dq_free = dq_full + 1;
+  uint64_t* mma_done = dq_free + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Work unit: (batch, kv head, key tile), key tile 0 first (it sees the most
+  // query tiles under the causal mask).
+  const int n_kt = (p.N + kTileN - 1) / kTileN;
+  const int kt = blockIdx.x % n_kt;
+  const int bkv = blockIdx.x / n_kt;
+  const int b = bkv / p.Hkv;
+  const int kvh = bkv % p.Hkv;
+  const int g = p.Hq / p.Hkv;
+  const int j0 = kt * kTileN;
+  const int n_qt = (p.N + BR - 1) / BR;
+  const int qt_first = p.causal ? j0 / BR : 0;
+  const int per_head = n_qt - qt_first;
+  const int n_it = g * per_head;
+  const float c = p.scale_log2;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&st_full[s], 1 + 32);
+      mbar_init(&st_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(dp_full, 1);
+    mbar_init(dp_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(p_free, 1);
+    mbar_init(ds_full, 128);
+    mbar_init(ds_free, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx w{abort_flag, p.status, p.wait_budget_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    regs_dec<kBwdRegsControl, kBwdRegsLaunch>();
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(kv_full, 2 * C::kKVBytes);
+#pragma unroll
+      for (int z = 0; z < D / 64; ++z) {
+        tma_load_3d(smem + C::kOffK + z * C::kKVRegion, &tmK, kv_full, z * 64, j0, bkv);
+        tma_load_3d(smem + C::kOffV + z * C::kKVRegion, &tmV, kv_full, z * 64, j0, bkv);
+      }
+    }
+    bool ok = true;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int s = it % ST;
+      const int h = kvh * g + it / per_head;
+      const int i0 = (qt_first + it % per_head) * BR;
+      const int q_head = b * p.Hq + h;
+      ok = mbar_wait(&st_empty[s], ((it / ST) & 1) ^ 1, w);
+      if (!ok) break;
+      uint8_t* stage = smem + C::kOffStage + s * C::kStageBytes;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&st_full[s], 2 * C::kQBytes);
+#pragma unroll
+        for (int z = 0; z < D / 64; ++z) {
+          tma_load_3d(stage + z * C::kQRegion, &tmQ, &st_full[s], z * 64, i0, q_head);
+          tma_load_3d(stage + C::kQBytes + z * C::kQRegion, &tmDO, &st_full[s], z * 64, i0, q_head);
+        }
+      }
+      float* lse2 = reinterpret_cast<float*>(stage + 2 * C::kQBytes);
+      float* dl = lse2 + BR;
+      const size_t rbase = (size_t)q_head * p.N;
+#pragma unroll
+      for (int r = lane; r < BR; r += 32) {
+        const int i = i0 + r;
+        const bool in = i < p.N;
+        lse2[r] = in ? p.lse[rbase + i] * 1.4426950408889634f : INFINITY;
+        dl[r] = in ? p.delta[rbase + i] : 0.f;
+      }
+      mbar_arrive(&st_full[s]);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    regs_dec<kBwdRegsControl, kBwdRegsLaunch>();
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, BR, false, false);   // S^T, dP^T
+      constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, false, true);    // dV, dK
+      constexpr uint32_t kIdQ = idesc_bf16_f32(128, 64, true, true);     // dQ (or dQ^T)
+      const uint32_t k_base = smem_u32(smem + C::kOffK);
+      const uint32_t v_base = smem_u32(smem + C::kOffV);
+      const uint32_t st_base = smem_u32(smem + C::kOffStage);
+      const uint32_t pt_base = smem_u32(smem + C::kOffP);
+      const uint32_t ds_base = smem_u32(smem + C::kOffDS);
+      // X^T = A B^T over the head dim: A = K or V tile, B = Q or dO tile (both K-major)
+      auto mma_scores = [&](uint32_t a_base, uint32_t b_base, uint32_t col) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t a = sdesc_sw128(a_base + (k >> 2) * C::kKVRegion + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b_base + (k >> 2) * C::kQRegion + (k & 3) * 32, 16, 1024);
+          mma_bf16_ss(tmem + col, a, bd, kIdS, k > 0 ? 1u : 0u);
+        }
+      };
+      // acc += A B over the query rows: A = P^T or dS^T (K-major), B = dO or Q (MN-major)
+      auto mma_accum = [&](uint32_t a_base, uint32_t b_base, uint32_t col, bool first) {
+#pragma unroll
+        for (int k = 0; k < BR / 16; ++k) {
+          const uint64_t a = sdesc_sw128(a_base + (k >> 2) * C::kPRegion + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b_base + k * 2048, C::kQRegion, 1024);
+          mma_bf16_ss(tmem + col, a, bd, kIdKV, (!first || k > 0) ? 1u : 0u);
+        }
+      };
+      // dQ (d = 64): A = dS (MN-major view of dS^T), B = K (MN-major), over the 128 keys.
+      // dQ^T (d = 128): A = K^T (MN-major view of K), B = dS^T (MN-major), over the 128 keys.
+      auto mma_dq = [&]() {
+#pragma unroll
+        for (int k = 0; k < kTileN / 16; ++k) {
+          uint64_t a, bd;
+          if (D == 128) {
+            a = sdesc_sw128(k_base + k * 2048, C::kKVRegion, 1024);
+            bd = sdesc_sw128(ds_base + k * 2048, C::kPRegion, 1024);
+          } else {
+            a = sdesc_sw128(ds_base + k * 2048, C::kPRegion, 1024);
+            bd = sdesc_sw128(k_base + k * 2048, C::kKVRegion, 1024);
+          }
+          mma_bf16_ss(tmem + C::kColDQ, a, bd, kIdQ, k > 0 ? 1u : 0u);
+        }
+      };
+      auto stage_addr = [&](int it) { return st_base + (it % ST) * C::kStageBytes; };
+      bool ok = mbar_wait(kv_full, 0, w);
+      if (ok && n_it > 0) ok = mbar_wait(&st_full[0], 0, w);
+      tc_fence_after();
+      if (ok && n_it > 0) {
+        mma_scores(k_base, stage_addr(0), C::kColS);
+        mma_commit(s_full);
+        mma_scores(v_base, stage_addr(0) + C::kQBytes, C::kColDP);
+        mma_commit(dp_full);
+      }
+      for (int it = 0; it < n_it && ok; ++it) {
+        const uint32_t sa = stage_addr(it);
+        const uint32_t ph = it & 1;
+        // dV += P^T dO_i
+        if (!(ok = mbar_wait(p_full, ph, w))) break;
+        tc_fence_after();
+        mma_accum(pt_base, sa + C::kQBytes, C::kColDV, it == 0);
+        mma_commit(p_free);
+        // next scores as early as possible
+        if (it + 1 < n_it) {
+          if (!(ok = mbar_wait(&st_full[(it + 1) % ST], ((it + 1) / ST) & 1, w))) break;
+          if (!(ok = mbar_wait(s_free, ph, w))) break;
+          tc_fence_after();
+          mma_scores(k_base, stage_addr(it + 1), C::kColS);
+          mma_commit(s_full);
+        }
+        // dK += dS^T Q_i ; dQ_i
+        if (!(ok = mbar_wait(ds_full, ph, w))) break;
+        tc_fence_after();
+        mma_accum(ds_base, sa, C::kColDK, it == 0);
+        if (it >= 1 && !(ok = mbar_wait(dq_free, ph ^ 1, w))) break;
+        tc_fence_after();
+        mma_dq();
+        mma_commit(dq_full);
+        mma_commit(ds_free);
+        mma_commit(&st_empty[it % ST]);
+        if (it + 1 < n_it) {
+          if (!(ok = mbar_wait(dp_free, ph, w))) break;
+          tc_fence_after();
+          mma_scores(v_base, stage_addr(it + 1) + C::kQBytes, C::kColDP);
+          mma_commit(dp_full);
+        }
+      }
+      mma_commit(mma_done);
+      WaitCtx drain{abort_flag, p.status, 20000000ull};
+      volatile int zero = 0;
+      drain.abort_flag = &zero;
+      mbar_wait(mma_done, 0, drain);
+    }
+  } else if (warp < 4) {
+    regs_dec<kBwdRegsControl, kBwdRegsLaunch>();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ P^T and dS^T
+    regs_inc<kBwdRegsSoftmax, kBwdRegsLaunch>();
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // key row within the tile
+    const int key = j0 + row;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t pt_tile = smem_u32(smem + C::kOffP);
+    const uint32_t ds_tile = smem_u32(smem + C::kOffDS);
+    const bool key_valid = key < p.N;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % ST;
+      const uint32_t ph = it & 1;
+      const int i0 = (qt_first + it % per_head) * BR;
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::kOffStage + s * C::kStageBytes + 2 * C::kQBytes);
+      const float* dl = lse2 + BR;
+      if (!mbar_wait(&st_full[s], (it / ST) & 1, w)) break;
+      if (!mbar_wait(s_full, ph, w)) break;
+      tc_fence_after();
+      float pr[BR];
+#pragma unroll
+      for (int cc = 0; cc < BR / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + C::kColS + cc * 32, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pr[cc * 32 + i] = __uint_as_float(r[i]);
+      }
+      tc_fence_before();
+      mbar_arrive(s_free);
+      // P^T[key][q] = 2^(S c - LSE2_q), zero for future queries and invalid keys.
+      const bool diag = p.causal && i0 < j0 + kTileN;
+#pragma unroll
+      for (int i = 0; i < BR; ++i) {
+        float e = ex2(fmaf(pr[i], c, -lse2[i]));
+        if (diag && i0 + i < key) e = 0.f;
+        pr[i] = key_valid ? e : 0.f;
+      }
+      if (it >= 1 && !mbar_wait(p_free, ph ^ 1, w)) break;
+#pragma unroll
+      for (int ch = 0; ch < BR / 8; ++ch) {
+        const int c0 = ch * 8;
+        st_shared_v4(pt_tile + (ch >> 3) * C::kPRegion + sw128_offset(row, ch & 7),
+                     pack_bf16x2(pr[c0], pr[c0 + 1]), pack_bf16x2(pr[c0 + 2], pr[c0 + 3]),
+                     pack_bf16x2(pr[c0 + 4], pr[c0 + 5]), pack_bf16x2(pr[c0 + 6], pr[c0 + 7]));
+      }
+      fence_async_smem();
+      mbar_arrive(p_full);
+      // dS^T = P^T o (dP^T - D_q)
+      if (!mbar_wait(dp_full, ph, w)) break;
+      if (it >= 1 && !mbar_wait(ds_free, ph ^ 1, w)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < BR / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + C::kColDP + cc * 32, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t u[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const int i = cc * 32 + ch * 8 + e2 * 2;
+            const int ri = ch * 8 + e2 * 2;
+            const float a = pr[i] * (__uint_as_float(r[ri]) - dl[i]);
+            const float bb = pr[i + 1] * (__uint_as_float(r[ri + 1]) - dl[i + 1]);
+            u[e2] = pack_bf16x2(a, bb);
+          }
+          const int chunk = cc * 4 + ch;
+          st_shared_v4(ds_tile + (chunk >> 3) * C::kPRegion + sw128_offset(row, chunk & 7), u[0], u[1], u[2],
+                       u[3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(dp_free);
+      fence_async_smem();
+      mbar_arrive(ds_full);
+    }
+  } else {
+    // ------------------------------------------------------------ dQ reductions, dK / dV epilogue
+    const int quarter = warp & 3;
+    const int tl = quarter * 32 + lane;  // TMEM lane
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int h = kvh * g + it / per_head;
+      const int i0 = (qt_first + it % per_head) * BR;
+      const size_t head_row0 = (size_t)(b * p.Hq + h) * p.N;
+      if (!(ok = mbar_wait(dq_full, it & 1, w))) break;
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tmem + lane_off + C::kColDQ, r0);
+      tmem_ld_wait(r0);
+      tmem_ld32(tmem + lane_off + C::kColDQ + 32, r1);
+      tmem_ld_wait(r1);
+      tc_fence_before();
+      mbar_arrive(dq_free);
+      if (D == 128) {
+        // lane = head-dim column, TMEM columns = the BR = 64 query rows
+        float* base = p.dq_acc + (head_row0 + i0) * D + tl;
+        const int nq = min(64, p.N - i0);
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          if (q < nq) red_add(base + (size_t)q * D, __uint_as_float(r0[q]));
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          if (q + 32 < nq) red_add(base + (size_t)(q + 32) * D, __uint_as_float(r1[q]));
+      } else {
+        // lane = query row, TMEM columns = the 64 head-dim columns
+        if (i0 + tl < p.N) {
+          float* base = p.dq_acc + (head_row0 + i0 + tl) * D;
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            red_add_v4(base + v * 4, __uint_as_float(r0[v * 4]), __uint_as_float(r0[v * 4 + 1]),
+                       __uint_as_float(r0[v * 4 + 2]), __uint_as_float(r0[v * 4 + 3]));
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            red_add_v4(base + 32 + v * 4, __uint_as_float(r1[v * 4]), __uint_as_float(r1[v * 4 + 1]),
+                       __uint_as_float(r1[v * 4 + 2]), __uint_as_float(r1[v * 4 + 3]));
+        }
+      }
+    }
+    if (ok && n_it > 0 && mbar_wait(mma_done, 0, w)) {
+      tc_fence_after();
+      // dK, dV rows: TMEM lane = key row
+      const int key = j0 + tl;
+      const bool valid = key < p.N;
+      const size_t row_idx = (size_t)bkv * p.N + key;
+      uint4* dk_dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + row_idx * D);
+      uint4* dv_dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + row_idx * D);
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which ? C::kColDK : C::kColDV;
+        const float mul = which ? p.scale : 1.f;
+        uint4* dst = which ? dk_dst : dv_dst;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + col + cc * 32, r);
+          tmem_ld_wait(r);
+          if (valid) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const int i = v4 * 8;
+              uint4 u;
+              u.x = pack_bf16x2(__uint_as_float(r[i]) * mul, __uint_as_float(r[i + 1]) * mul);
+              u.y = pack_bf16x2(__uint_as_float(r[i + 2]) * mul, __uint_as_float(r[i + 3]) * mul);
+              u.z = pack_bf16x2(__uint_as_float(r[i + 4]) * mul, __uint_as_float(r[i + 5]) * mul);
+              u.w = pack_bf16x2(__uint_as_float(r[i + 6]) * mul, __uint_as_float(r[i + 7]) * mul);
+              dst[cc * 4 + v4] = u;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                         const BwdParams& p, cudaStream_t s) {
+  using C = BwdCfg<D>;
+  static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+  const long long rows = (long long)p.B * p.Hq * p.N;
+  const int blocks = (int)std::min<long long>((rows * (D / 8) + 255) / 256, 8LL * sm_count());
+  bwd_preprocess_kernel<D><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(p.o),
+                                                   static_cast<const __nv_bfloat16*>(p.dout), p.delta, p.dq_acc, rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const long long grid = (long long)p.B * p.Hkv * ((p.N + kTileN - 1) / kTileN);
+  bwd_main_kernel<D><<<(unsigned)grid, kBwdThreads, C::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long n8 = rows * D / 8;
+  const int cblocks = (int)std::min<long long>((n8 + 255) / 256, 8LL * sm_count());
+  bwd_convert_kernel<<<cblocks, 256, 0, s>>>(p.dq_acc, static_cast<__nv_bfloat16*>(p.dq), n8, p.scale);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const BwdParams& p, cudaStream_t s) {
+  return p.d == 128 ? launch_bwd_d<128>(tq, tk, tv, tdo, p, s) : launch_bwd_d<64>(tq, tk, tv, tdo, p, s);
+}
+
 }  // namespace fa

@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const WaitCtx w{abort_flag, p.status, p.wait_budget_ns};
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    regs_dec<kRegsControl>();
+    regs_dec<kRegsControl, kRegsLaunch>();
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    regs_dec<kRegsControl>();
+    regs_dec<kRegsControl, kRegsLaunch>();
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, false, true);
@@ -249,10 +249,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_wait(mma_final, 0, drain);
     }
   } else if (warp < 4) {
-    regs_dec<kRegsControl>();
+    regs_dec<kRegsControl, kRegsLaunch>();
   } else {
     // ------------------------------------------------------------ softmax
-    regs_inc<kRegsSoftmax>();
+    regs_inc<kRegsSoftmax, kRegsLaunch>();
     const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;

@@ -242,14 +242,18 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 
 // ----------------------------------------------------------------------------
 // register reallocation between warpgroups (all warps of a warpgroup execute
-// the same one). The shares must add up to the launch's threads x registers.
+// the same one). The shares must add up to at most the launch's threads x
+// registers. .dec must lower and .inc must raise the count the warp holds
+// (the launch count, `kLaunch`); anything else is undefined, hence the checks.
 // ----------------------------------------------------------------------------
-template <int N>
+template <int N, int kLaunch>
 __device__ __forceinline__ void regs_dec() {
+  static_assert(N % 8 == 0 && N >= 24 && N < kLaunch, "setmaxnreg.dec must lower the register count");
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
-template <int N>
+template <int N, int kLaunch>
 __device__ __forceinline__ void regs_inc() {
+  static_assert(N % 8 == 0 && N <= 256 && N > kLaunch, "setmaxnreg.inc must raise the register count");
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
