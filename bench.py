@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of the exact IO-aware attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload c3]
+
+One step is one pass of the whole path over one batch of synthetic input: the
+forward (O and LSE) and the backward (D, recomputation with dK/dV/dQ
+accumulation, dQ conversion). The default workload is B=2, H=32, N=8192,
+d=128, causal, bf16. It is the shape on which the pages' long-context claims
+and the forward/backward utilisation targets are stated (N >= 8K, d = 128,
+forward and backward). FLOPs are algorithmic: 4 B H N^2 d for the forward,
+halved for causal; 2.5x that for the backward.
+
+Rank 0 prints one JSON line. `value` is the whole-job TFLOP/s over all ranks
+(weak scaling: every rank runs its own replica of the workload; there is no
+data-path collective). `e2e` repeats the measurement with each step's inputs
+copied from pinned host memory and the results copied back inside the timed
+region. `roofline` reports the dominant kernel against the measured dense bf16
+peak. `cpu_baseline` times the float64 oracle on a bounded sample on the host
+cores. `--impl reference` times that oracle alone as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s on 1 B200 and % of dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+# DRAM bytes (read + write) per launch of the dominant kernel from one ncu
+# capture, with the hash of the kernel source it was taken on. A changed
+# source makes the figure stale and the bench reports null.
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    fname = {"bwd_main": "fa_bwd_sm100.cu", "fwd": "fa_fwd_sm100.cu"}[kernel]
+    paths = [os.path.join(ROOT, "exact_io_aware_44_b200", "csrc", f) for f in (fname, "sm100.cuh")]
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, group=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    backend = dist.get_backend(group)
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
+def barrier(group=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier(group=group)
+
+
+def job_throughput(flops_per_step_per_rank: float, world: int, max_seconds_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank's work over the slowest rank's time."""
+    return flops_per_step_per_rank * world / max_seconds_per_step / 1e12
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, interval_ms: int = 100):
+        self.gpu = gpu_index
+        self.interval = interval_ms
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms={self.interval}"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        rows = list(csv.reader(io.StringIO(open(self.path).read())))
+        os.unlink(self.path)
+        sm, mx, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                power.append(float(r[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock samples"]}
+        # samples under load: power well above idle
+        hi = [s for s, p in zip(sm, power) if p >= 0.5 * max(power)] or sm
+        return {"sm_mhz": statistics.median(hi), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the float64 oracle on a bounded sample of the workload
+# ---------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_head_step(w, b: int, h: int):
+    """Forward + backward of one (batch, head) of workload `w` in float64; returns FLOPs."""
+    import numpy as np
+    import oracle
+    import synth
+    q = synth.head_slice(w, synth.TID_Q, b, h)[None, None]
+    k = synth.head_slice(w, synth.TID_K, b, h // w.group)[None, None]
+    v = synth.head_slice(w, synth.TID_V, b, h // w.group)[None, None]
+    do = synth.head_slice(w, synth.TID_DO, b, h)[None, None]
+    t0 = time.perf_counter()
+    o, lse = oracle.attention_fwd64(q, k, v, w.causal, w.scale)
+    oracle.attention_bwd64(q, k, v, do, w.causal, w.scale, o=o, lse=lse)
+    dt = time.perf_counter() - t0
+    f = 4.0 * w.N * w.N * w.d * (0.5 if w.causal else 1.0)
+    return dt, f * (3.5 if w.backward else 1.0)
+
+
+def cpu_baseline(w, budget_s: float = 15.0):
+    total_t, total_f, heads = 0.0, 0.0, 0
+    while heads < w.B * w.Hq and (heads == 0 or total_t < budget_s):
+        b, h = divmod(heads, w.Hq)
+        dt, f = oracle_head_step(w, b, h)
+        total_t += dt
+        total_f += f
+        heads += 1
+    return {"value": total_f / total_t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{heads} of {w.B * w.Hq} (batch, head) pairs, full forward + backward each, float64 NumPy",
+            "seconds": round(total_t, 3)}
+
+
+# ---------------------------------------------------------------------------
+# our path
+# ---------------------------------------------------------------------------
+
+def run_ours(args, w, world, rank, local):
+    import numpy as np
+    import torch
+
+    import exact_io_aware_44_b200 as fa
+    import synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_budget)
+
+    # inputs: generated on the host (seeded), kept pinned for the e2e leg
+    host = {}
+    for name, tid in (("q", synth.TID_Q), ("k", synth.TID_K), ("v", synth.TID_V), ("do", synth.TID_DO)):
+        host[name] = torch.from_numpy(synth.tensor(w, tid)).to(torch.bfloat16).pin_memory()
+    d_in = {n: t.to(dev) for n, t in host.items()}
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    o = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    dq = torch.empty_like(o)
+    dk = torch.empty((B, Hkv, N, d), dtype=torch.bfloat16, device=dev)
+    dv = torch.empty_like(dk)
+    ws = torch.empty(fa.workspace_bytes(B, Hq, Hkv, N, d), dtype=torch.uint8, device=dev)
+    P = lambda t: t.data_ptr()
+
+    def step(events=None):
+        if events is not None:
+            events[0].record(stream)
+        rc = fa.fwd_raw(P(d_in["q"]), P(d_in["k"]), P(d_in["v"]), P(o), P(lse), B, Hq, Hkv, N, d, w.causal,
+                        w.scale, sp)
+        if rc:
+            raise fa.FAError(rc, "fa_fwd")
+        if not w.backward:
+            if events is not None:
+                for e in events[1:]:
+                    e.record(stream)
+            return
+        between = None
+        if events is not None:
+            between = lambda i: events[1 + i].record(stream)
+        rc = fa.bwd_phases_raw(P(d_in["q"]), P(d_in["k"]), P(d_in["v"]), P(o), P(lse), P(d_in["do"]), P(dq), P(dk),
+                               P(dv), P(ws), B, Hq, Hkv, N, d, w.causal, w.scale, sp, between=between)
+        if rc:
+            raise fa.FAError(rc, "fa_bwd")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = fa.get_status()
+    if st:
+        raise fa.FAError(st, "warm-up")
+
+    # ---------------------------------------------------- device-timed region
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(K):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    st = fa.get_status()
+    if st:
+        raise fa.FAError(st, "timed region")
+    ms_total = t_start.elapsed_time(t_end)
+    ms_step = reduce_max(ms_total / K)
+    # events: 0 fwd start, 1 bwd pre start (= fwd end), 2 main start, 3 convert start, 4 bwd end
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    pre_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    conv_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
+    f_fwd, f_bwd = w.fwd_flops(), (w.bwd_flops() if w.backward else 0.0)
+    value = job_throughput(f_fwd + f_bwd, world, ms_step / 1e3)
+
+    kernels = {
+        "fwd": {"ms": fwd_ms, "tflops": f_fwd / fwd_ms / 1e9},
+        "bwd_preprocess": {"ms": pre_ms},
+        "bwd_main": {"ms": main_ms, "tflops": f_bwd / main_ms / 1e9 if main_ms > 0 else 0.0},
+        "bwd_convert": {"ms": conv_ms},
+    }
+    dominant = max(("fwd", "bwd_main"), key=lambda k: kernels[k]["ms"])
+    achieved = kernels[dominant]["tflops"]
+    traffic = None
+    rec = NCU_TRAFFIC.get((dominant, w.name))
+    if rec and rec.get("csrc_sha") == kernel_source_hash(dominant):
+        traffic = rec["bytes_per_launch"]
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": UNIT,
+                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": dominant,
+                "peak_source": f"{peak_src} dense bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
+                if peak_src == "measured" else "fallback 1.59 PFLOP/s",
+                "frac_of_sustained": round(achieved / float(peaks.get("bf16_tflops_sustained", peak)), 4)}
+
+    # ---------------------------------------------------- end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        out_host = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                    for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+        dev_out = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+        Ke = max(1, min(K, args.e2e_steps))
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(Ke):
+            for n in host:
+                d_in[n].copy_(host[n], non_blocking=True)
+            step()
+            for n in out_host:
+                out_host[n].copy_(dev_out[n], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = reduce_max(e0.elapsed_time(e1) / Ke)
+        e2e = {"value": round(job_throughput(f_fwd + f_bwd, world, e_ms / 1e3), 2), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 3),
+               "steps": Ke}
+        st = fa.get_status()
+        if st:
+            raise fa.FAError(st, "e2e region")
+
+    clk = clocks.summary()
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} "
+                               f"{'causal' if w.causal else 'non-causal'} bf16 "
+                               f"{'fwd+bwd' if w.backward else 'fwd'}",
+                   "B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "causal": w.causal,
+                   "l2": "inputs larger than L2 (Q, K, V, O, dO are "
+                         f"{B * Hq * N * d * 2 / 1e6:.0f} MB each; L2 is 126 MB)",
+                   "parallelism": f"replicas x{world}"},
+        "pct_of_peak": round(100 * value / world / peak, 2),
+        "fwd_tflops": round(kernels["fwd"]["tflops"], 1),
+        "bwd_tflops": round(f_bwd / (pre_ms + main_ms + conv_ms) / 1e9, 1) if w.backward else None,
+        "kernels_ms": {k: round(v["ms"], 4) for k, v in kernels.items()},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": (4 if w.backward else 1) * K,
+        "clocks": clk,
+    }
+    return result
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the float64 oracle as it stands, on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args, w):
+    times, flops = [], 0.0
+    n_heads = w.B * w.Hq
+    for i in range(args.warmup + args.steps):
+        b, h = divmod(i % n_heads, w.Hq)
+        dt, f = oracle_head_step(w, b, h)
+        if i >= args.warmup:
+            times.append(dt)
+            flops = f
+    ms = 1e3 * statistics.mean(times)
+    value = flops / (ms / 1e3) / 1e12
+    sample = f"one (batch, head) pair per step: full forward + backward of B=1 H=1 N={w.N} d={w.d} in float64"
+    return {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": 0, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} "
+                                   f"{'causal' if w.causal else 'non-causal'} fwd+bwd (sampled per step)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": blas_threads(),
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c3", help="c2, c3, c4 (forward only) or c5")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    world, rank, local = dist_env()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    try:
+        res = run_ours(args, w, world, rank, local)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

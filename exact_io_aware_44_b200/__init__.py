@@ -18,7 +18,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["fwd", "bwd", "fwd_raw", "bwd_raw", "workspace_bytes", "get_status", "set_wait_budget_ns",
+__all__ = ["fwd", "bwd", "fwd_raw", "bwd_raw", "bwd_phases_raw", "workspace_bytes", "get_status", "set_wait_budget_ns",
            "selftest_wait_timeout", "FAError", "LIB_PATH", "lib", "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
@@ -35,6 +35,9 @@ SIGNATURES = {
     "fa_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_bwd_preprocess": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "fa_bwd_main": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_bwd_convert": (_I, [_P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "fa_get_status": (_I, [_P]),
     "fa_set_wait_budget_ns": (None, [ctypes.c_uint64]),
     "fa_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
@@ -140,6 +143,29 @@ def bwd_raw(q, k, v, o, lse, do, dq, dk, dv, ws, B, Hq, Hkv, N, d, causal, scale
     """The C call itself on raw device pointers (ints); returns the status code."""
     return lib.fa_bwd(_P(q), _P(k), _P(v), _P(o), _P(lse), _P(do), _P(dq), _P(dk), _P(dv), _P(ws), B, Hq, Hkv, N,
                       d, int(bool(causal)), float(scale), _P(stream_ptr))
+
+
+def bwd_phases_raw(q, k, v, o, lse, do, dq, dk, dv, ws, B, Hq, Hkv, N, d, causal, scale, stream_ptr,
+                   between=None):
+    """fa_bwd as its three C calls (preprocess, main, convert) on raw pointers.
+    `between(i)` (optional) is called before phase i = 0, 1, 2 and after the
+    last (i = 3), e.g. to record CUDA events on the same stream. Returns the
+    first nonzero status code, else 0."""
+    c = int(bool(causal))
+    st = _P(stream_ptr)
+    calls = (lambda: lib.fa_bwd_preprocess(_P(o), _P(do), _P(ws), B, Hq, Hkv, N, d, st),
+             lambda: lib.fa_bwd_main(_P(q), _P(k), _P(v), _P(lse), _P(do), _P(dk), _P(dv), _P(ws), B, Hq, Hkv, N, d,
+                                     c, float(scale), st),
+             lambda: lib.fa_bwd_convert(_P(dq), _P(ws), B, Hq, Hkv, N, d, float(scale), st))
+    for i, call in enumerate(calls):
+        if between is not None:
+            between(i)
+        rc = call()
+        if rc != 0:
+            return rc
+    if between is not None:
+        between(3)
+    return 0
 
 
 def bwd(q, k, v, o, lse, do, causal: bool = True, scale: float | None = None, workspace=None, out=None,

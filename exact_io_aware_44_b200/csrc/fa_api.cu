@@ -199,27 +199,44 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   return delta + rows * (size_t)d * sizeof(float);
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
-           void* dk, void* dv, void* workspace, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
-           void* stream) {
+}  // extern "C"
+
+namespace fa {
+namespace {
+
+enum BwdPhase { kPhasePre = 1, kPhaseMain = 2, kPhaseConvert = 4, kPhaseAll = 7 };
+
+// Validates the arguments each requested phase reads, then launches the phases
+// in order on `stream`. Nothing is launched unless every check passes.
+int run_bwd(int phases, const void* q, const void* k, const void* v, const void* o, const float* lse,
+            const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv, int N, int d,
+            int causal, float scale, void* stream) {
   bool empty;
   int rc = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
   if (rc != FA_OK) return rc;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (empty) return FA_OK;
-  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return FA_ERR_ALIGNMENT;
+  const bool pre = phases & kPhasePre, main = phases & kPhaseMain, conv = phases & kPhaseConvert;
+  if (!workspace) return FA_ERR_INVALID_ARG;
+  if (pre && (!o || !dout)) return FA_ERR_INVALID_ARG;
+  if (main && (!q || !k || !v || !lse || !dout || !dk || !dv)) return FA_ERR_INVALID_ARG;
+  if (conv && !dq) return FA_ERR_INVALID_ARG;
+  const void* need16[] = {pre ? o : nullptr,     pre || main ? dout : nullptr, main ? q : nullptr,
+                          main ? k : nullptr,    main ? v : nullptr,           main ? lse : nullptr,
+                          main ? dk : nullptr,   main ? dv : nullptr,          conv ? dq : nullptr};
+  for (const void* ptr : need16)
+    if (ptr && !aligned16(ptr)) return FA_ERR_ALIGNMENT;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_ALIGNMENT;
   DeviceInfo* di;
   if ((rc = current_device(&di)) != FA_OK) return rc;
   CUtensorMap tq, tk, tv, tdo;
-  const int q_rows = (d == 128) ? 64 : 128;  // query rows per backward tile
-  if ((rc = make_map(&tq, q, d, N, B * Hq, q_rows)) != FA_OK) return rc;
-  if ((rc = make_map(&tk, k, d, N, B * Hkv)) != FA_OK) return rc;
-  if ((rc = make_map(&tv, v, d, N, B * Hkv)) != FA_OK) return rc;
-  if ((rc = make_map(&tdo, dout, d, N, B * Hq, q_rows)) != FA_OK) return rc;
+  if (main) {
+    const int q_rows = (d == 128) ? 64 : 128;  // query rows per backward tile
+    if ((rc = make_map(&tq, q, d, N, B * Hq, q_rows)) != FA_OK) return rc;
+    if ((rc = make_map(&tk, k, d, N, B * Hkv)) != FA_OK) return rc;
+    if ((rc = make_map(&tv, v, d, N, B * Hkv)) != FA_OK) return rc;
+    if ((rc = make_map(&tdo, dout, d, N, B * Hq, q_rows)) != FA_OK) return rc;
+  }
   const size_t rows = (size_t)B * Hq * N;
   const size_t delta_bytes = (rows * sizeof(float) + 255) & ~size_t(255);
   BwdParams p;
@@ -244,8 +261,39 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_budget_ns = g_wait_budget_ns.load();
-  if (launch_bwd_bf16(tq, tk, tv, tdo, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pre && launch_bwd_preprocess(p, s) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (main && launch_bwd_main(tq, tk, tv, tdo, p, s) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (conv && launch_bwd_convert(p, s) != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+           void* dk, void* dv, void* workspace, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+           void* stream) {
+  return run_bwd(kPhaseAll, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, causal, scale, stream);
+}
+
+int fa_bwd_preprocess(const void* o, const void* dout, void* workspace, int B, int Hq, int Hkv, int N, int d,
+                      void* stream) {
+  return run_bwd(kPhasePre, nullptr, nullptr, nullptr, o, nullptr, dout, nullptr, nullptr, nullptr, workspace, B, Hq,
+                 Hkv, N, d, 0, 1.f, stream);
+}
+
+int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk, void* dv,
+                void* workspace, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  return run_bwd(kPhaseMain, q, k, v, nullptr, lse, dout, nullptr, dk, dv, workspace, B, Hq, Hkv, N, d, causal, scale,
+                 stream);
+}
+
+int fa_bwd_convert(void* dq, const void* workspace, int B, int Hq, int Hkv, int N, int d, float scale, void* stream) {
+  return run_bwd(kPhaseConvert, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dq, nullptr, nullptr,
+                 const_cast<void*>(workspace), B, Hq, Hkv, N, d, 0, scale, stream);
 }
 
 int fa_get_status(void* stream) {

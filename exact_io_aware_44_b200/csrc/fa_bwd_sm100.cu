@@ -20,14 +20,19 @@
 //                     then added to the fp32 accumulator with red.global.add.
 //   bwd_convert     dQ = bf16(scale * accumulator).
 //
-// bwd_main roles (384 threads):
+// bwd_main roles (512 threads):
 //   warp 0      producer: K, V once (TMA); per query tile Q_i, dO_i (TMA) and
 //               LSE_i log2(e), D_i (plain loads) into a ring of stages.
 //   warp 1      allocates TMEM; one lane issues every tcgen05.mma.
-//   warps 4-7   thread = key row: P^T and dS^T, written to shared memory in the
-//               128-byte-swizzled K-major layout.
-//   warps 8-11  thread = TMEM lane of the dQ tile: reads it and issues the fp32
+//   warps 4-11  two warpgroups, thread = key row; warpgroup h computes P^T and
+//               dS^T for query columns [h BR/2, (h+1) BR/2) and writes them to
+//               shared memory in the 128-byte-swizzled K-major layout.
+//   warps 12-15 thread = TMEM lane of the dQ tile: reads it and issues the fp32
 //               reductions; at the end, writes dK and dV.
+//
+// MMA issue order per query tile i: dV(i), S(i+1), dP(i+1), dK(i), dQ(i). The
+// next tile's scores and dP are computed while the elementwise warpgroups
+// still work on dS(i) and P(i+1), so the tensor core always has queued work.
 //
 // Query tiles are BR = 64 rows for d = 128 (so dQ^T = K^T dS^T has M = d = 128)
 // and BR = 128 rows for d = 64 (so dQ = dS K has M = 128 query rows). TMEM
@@ -43,14 +48,14 @@
 namespace fa {
 namespace {
 
-constexpr int kBwdThreads = 384;
-// Register split: the launch gives 168 per thread (384 x 168 = 64512). The
-// control warpgroup lowers to 56, the P/dS warpgroup raises to 232, and the dQ
-// warpgroup keeps the launch count: 128 x (56 + 232 + 168) = 58368 <= 64512.
-constexpr int kBwdRegsLaunch = 168;
+constexpr int kBwdThreads = 512;
+// Register split: the launch gives 128 per thread (512 x 128 = 65536). The
+// control warpgroup lowers to 56, the two P/dS warpgroups raise to 160, and
+// the dQ warpgroup keeps the launch count: 128 x (56 + 2 x 160 + 128) = 64512.
+constexpr int kBwdRegsLaunch = 128;
 constexpr int kBwdRegsControl = 56;
-constexpr int kBwdRegsSoftmax = 232;
-static_assert(128 * (kBwdRegsControl + kBwdRegsSoftmax + kBwdRegsLaunch) <= kBwdThreads * kBwdRegsLaunch,
+constexpr int kBwdRegsSoftmax = 160;
+static_assert(128 * (kBwdRegsControl + 2 * kBwdRegsSoftmax + kBwdRegsLaunch) <= kBwdThreads * kBwdRegsLaunch,
               "register split");
 
 template <int D>
@@ -207,12 +212,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&st_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
+    mbar_init(s_free, 256);
     mbar_init(dp_full, 1);
-    mbar_init(dp_free, 128);
-    mbar_init(p_full, 128);
+    mbar_init(dp_free, 256);
+    mbar_init(p_full, 256);
     mbar_init(p_free, 1);
-    mbar_init(ds_full, 128);
+    mbar_init(ds_full, 256);
     mbar_init(ds_free, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 128);
@@ -338,13 +343,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         mma_accum(pt_base, sa + C::kQBytes, C::kColDV, it == 0);
         mma_commit(p_free);
-        // next scores as early as possible
+        // the next tile's S^T and dP^T, as soon as their TMEM buffers were read
         if (it + 1 < n_it) {
           if (!(ok = mbar_wait(&st_full[(it + 1) % ST], ((it + 1) / ST) & 1, w))) break;
           if (!(ok = mbar_wait(s_free, ph, w))) break;
           tc_fence_after();
           mma_scores(k_base, stage_addr(it + 1), C::kColS);
           mma_commit(s_full);
+          if (!(ok = mbar_wait(dp_free, ph, w))) break;
+          tc_fence_after();
+          mma_scores(v_base, stage_addr(it + 1) + C::kQBytes, C::kColDP);
+          mma_commit(dp_full);
         }
         // dK += dS^T Q_i ; dQ_i
         if (!(ok = mbar_wait(ds_full, ph, w))) break;
@@ -356,12 +365,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_commit(dq_full);
         mma_commit(ds_free);
         mma_commit(&st_empty[it % ST]);
-        if (it + 1 < n_it) {
-          if (!(ok = mbar_wait(dp_free, ph, w))) break;
-          tc_fence_after();
-          mma_scores(v_base, stage_addr(it + 1) + C::kQBytes, C::kColDP);
-          mma_commit(dp_full);
-        }
       }
       mma_commit(mma_done);
       WaitCtx drain{abort_flag, p.status, 20000000ull};
@@ -371,9 +374,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp < 4) {
     regs_dec<kBwdRegsControl, kBwdRegsLaunch>();
-  } else if (warp < 8) {
-    // ------------------------------------------------------------ P^T and dS^T
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ P^T and dS^T (half the columns each)
     regs_inc<kBwdRegsSoftmax, kBwdRegsLaunch>();
+    constexpr int HB = BR / 2;  // query columns per warpgroup
+    const int half = (warp - 4) >> 2;
+    const int col0 = half * HB;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key row within the tile
     const int key = j0 + row;
@@ -384,17 +390,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int it = 0; it < n_it; ++it) {
       const int s = it % ST;
       const uint32_t ph = it & 1;
-      const int i0 = (qt_first + it % per_head) * BR;
-      const float* lse2 = reinterpret_cast<const float*>(smem + C::kOffStage + s * C::kStageBytes + 2 * C::kQBytes);
+      const int i0 = (qt_first + it % per_head) * BR + col0;  // first query of this half
+      const float* lse2 =
+          reinterpret_cast<const float*>(smem + C::kOffStage + s * C::kStageBytes + 2 * C::kQBytes) + col0;
       const float* dl = lse2 + BR;
       if (!mbar_wait(&st_full[s], (it / ST) & 1, w)) break;
       if (!mbar_wait(s_full, ph, w)) break;
       tc_fence_after();
-      float pr[BR];
+      float pr[HB];
 #pragma unroll
-      for (int cc = 0; cc < BR / 32; ++cc) {
+      for (int cc = 0; cc < HB / 32; ++cc) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_off + C::kColS + cc * 32, r);
+        tmem_ld32(tmem + lane_off + C::kColS + col0 + cc * 32, r);
         tmem_ld_wait(r);
 #pragma unroll
         for (int i = 0; i < 32; ++i) pr[cc * 32 + i] = __uint_as_float(r[i]);
@@ -404,48 +411,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // P^T[key][q] = 2^(S c - LSE2_q), zero for future queries and invalid keys.
       const bool diag = p.causal && i0 < j0 + kTileN;
 #pragma unroll
-      for (int i = 0; i < BR; ++i) {
+      for (int i = 0; i < HB; ++i) {
         float e = ex2(fmaf(pr[i], c, -lse2[i]));
         if (diag && i0 + i < key) e = 0.f;
         pr[i] = key_valid ? e : 0.f;
       }
       if (it >= 1 && !mbar_wait(p_free, ph ^ 1, w)) break;
 #pragma unroll
-      for (int ch = 0; ch < BR / 8; ++ch) {
+      for (int ch = 0; ch < HB / 8; ++ch) {
         const int c0 = ch * 8;
-        st_shared_v4(pt_tile + (ch >> 3) * C::kPRegion + sw128_offset(row, ch & 7),
+        const int chunk = col0 / 8 + ch;
+        st_shared_v4(pt_tile + (chunk >> 3) * C::kPRegion + sw128_offset(row, chunk & 7),
                      pack_bf16x2(pr[c0], pr[c0 + 1]), pack_bf16x2(pr[c0 + 2], pr[c0 + 3]),
                      pack_bf16x2(pr[c0 + 4], pr[c0 + 5]), pack_bf16x2(pr[c0 + 6], pr[c0 + 7]));
       }
       fence_async_smem();
       mbar_arrive(p_full);
-      // dS^T = P^T o (dP^T - D_q)
+      // dS^T = P^T o (dP^T - D_q); dP^T is read out whole first so the next
+      // tile's dP^T can be issued at once.
       if (!mbar_wait(dp_full, ph, w)) break;
-      if (it >= 1 && !mbar_wait(ds_free, ph ^ 1, w)) break;
       tc_fence_after();
+      float dp[HB];
 #pragma unroll
-      for (int cc = 0; cc < BR / 32; ++cc) {
+      for (int cc = 0; cc < HB / 32; ++cc) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_off + C::kColDP + cc * 32, r);
+        tmem_ld32(tmem + lane_off + C::kColDP + col0 + cc * 32, r);
         tmem_ld_wait(r);
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t u[4];
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const int i = cc * 32 + ch * 8 + e2 * 2;
-            const int ri = ch * 8 + e2 * 2;
-            const float a = pr[i] * (__uint_as_float(r[ri]) - dl[i]);
-            const float bb = pr[i + 1] * (__uint_as_float(r[ri + 1]) - dl[i + 1]);
-            u[e2] = pack_bf16x2(a, bb);
-          }
-          const int chunk = cc * 4 + ch;
-          st_shared_v4(ds_tile + (chunk >> 3) * C::kPRegion + sw128_offset(row, chunk & 7), u[0], u[1], u[2],
-                       u[3]);
-        }
+        for (int i = 0; i < 32; ++i) dp[cc * 32 + i] = __uint_as_float(r[i]);
       }
       tc_fence_before();
       mbar_arrive(dp_free);
+      uint32_t dsp[HB / 2];
+#pragma unroll
+      for (int i = 0; i < HB; i += 2)
+        dsp[i / 2] = pack_bf16x2(pr[i] * (dp[i] - dl[i]), pr[i + 1] * (dp[i + 1] - dl[i + 1]));
+      if (it >= 1 && !mbar_wait(ds_free, ph ^ 1, w)) break;
+#pragma unroll
+      for (int ch = 0; ch < HB / 8; ++ch) {
+        const int chunk = col0 / 8 + ch;
+        st_shared_v4(ds_tile + (chunk >> 3) * C::kPRegion + sw128_offset(row, chunk & 7), dsp[ch * 4],
+                     dsp[ch * 4 + 1], dsp[ch * 4 + 2], dsp[ch * 4 + 3]);
+      }
       fence_async_smem();
       mbar_arrive(ds_full);
     }
@@ -548,33 +555,42 @@ int sm_count() {
 }
 
 template <int D>
-cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                         const BwdParams& p, cudaStream_t s) {
-  using C = BwdCfg<D>;
-  static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+cudaError_t launch_preprocess_d(const BwdParams& p, cudaStream_t s) {
   const long long rows = (long long)p.B * p.Hq * p.N;
   const int blocks = (int)std::min<long long>((rows * (D / 8) + 255) / 256, 8LL * sm_count());
   bwd_preprocess_kernel<D><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(p.o),
                                                    static_cast<const __nv_bfloat16*>(p.dout), p.delta, p.dq_acc, rows);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_main_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                          const BwdParams& p, cudaStream_t s) {
+  using C = BwdCfg<D>;
+  static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long grid = (long long)p.B * p.Hkv * ((p.N + kTileN - 1) / kTileN);
   bwd_main_kernel<D><<<(unsigned)grid, kBwdThreads, C::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const long long n8 = rows * D / 8;
-  const int cblocks = (int)std::min<long long>((n8 + 255) / 256, 8LL * sm_count());
-  bwd_convert_kernel<<<cblocks, 256, 0, s>>>(p.dq_acc, static_cast<__nv_bfloat16*>(p.dq), n8, p.scale);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_bwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+cudaError_t launch_bwd_preprocess(const BwdParams& p, cudaStream_t s) {
+  return p.d == 128 ? launch_preprocess_d<128>(p, s) : launch_preprocess_d<64>(p, s);
+}
+
+cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const BwdParams& p, cudaStream_t s) {
-  return p.d == 128 ? launch_bwd_d<128>(tq, tk, tv, tdo, p, s) : launch_bwd_d<64>(tq, tk, tv, tdo, p, s);
+  return p.d == 128 ? launch_main_d<128>(tq, tk, tv, tdo, p, s) : launch_main_d<64>(tq, tk, tv, tdo, p, s);
+}
+
+cudaError_t launch_bwd_convert(const BwdParams& p, cudaStream_t s) {
+  const long long n8 = (long long)p.B * p.Hq * p.N * p.d / 8;
+  const int blocks = (int)std::min<long long>((n8 + 255) / 256, 8LL * sm_count());
+  bwd_convert_kernel<<<blocks, 256, 0, s>>>(p.dq_acc, static_cast<__nv_bfloat16*>(p.dq), n8, p.scale);
+  return cudaGetLastError();
 }
 
 }  // namespace fa

@@ -49,8 +49,11 @@ struct BwdParams {
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int d, cudaStream_t s);
 cudaError_t launch_fwd_f32(const FwdF32Params& p, cudaStream_t s);
-cudaError_t launch_bwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+// Backward phases: D and zeroed dQ accumulator; main kernel; dQ conversion.
+cudaError_t launch_bwd_preprocess(const BwdParams& p, cudaStream_t s);
+cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const BwdParams& p, cudaStream_t s);
+cudaError_t launch_bwd_convert(const BwdParams& p, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* status, uint64_t budget_ns, cudaStream_t s);
 
 }  // namespace fa

@@ -117,6 +117,24 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * The three phases fa_bwd runs, in this order, on one stream. They exist so a
+ * caller (or a profiler) can time or interleave them; fa_bwd(...) is exactly
+ * fa_bwd_preprocess, then fa_bwd_main, then fa_bwd_convert with the same arguments.
+ *   fa_bwd_preprocess  D_i = sum_c dO_ic O_ic into the workspace, and zeroes
+ *                      the workspace's fp32 dQ accumulator.
+ *   fa_bwd_main        recomputes S and P per tile and accumulates dK, dV
+ *                      (written as bf16) and the fp32 dQ accumulator.
+ *   fa_bwd_convert     dq = bf16(scale * dQ accumulator).
+ * Arguments, layouts and error codes are those of fa_bwd; each phase only reads
+ * the pointers it needs (the others may be NULL).
+ */
+int fa_bwd_preprocess(const void* o, const void* dout, void* workspace, int B, int Hq, int Hkv, int N, int d,
+                      void* stream);
+int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dout, void* dk, void* dv,
+                void* workspace, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
+int fa_bwd_convert(void* dq, const void* workspace, int B, int Hq, int Hkv, int N, int d, float scale, void* stream);
+
+/*
  * fa_get_status -- synchronise `stream`, then return and clear the device
  * status word of the current device (FA_OK or the first device-side error
  * since the last call). Returns FA_ERR_LAUNCH if the stream reports a CUDA error.

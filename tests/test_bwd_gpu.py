@@ -114,3 +114,22 @@ def sampled_bwd_check(w, device):
 @pytest.mark.parametrize("name", ["c3", "c5"])
 def test_bf16_bwd_full_size_sampled(cuda_device, name):
     sampled_bwd_check(synth.WORKLOADS[name], cuda_device)
+
+
+def test_bwd_equals_its_three_phases(cuda_device):
+    """fa_bwd is fa_bwd_preprocess, fa_bwd_main and fa_bwd_convert in order."""
+    import torch
+    import exact_io_aware_44_b200 as fa
+    w = synth.small(1, 4, 2, 384, 128, True, seed=21)
+    q, k, v, do = (to_dev(synth.tensor(w, t), torch.bfloat16, cuda_device) for t in range(4))
+    o, lse = fa.fwd(q, k, v)
+    dq1, dk1, dv1 = fa.bwd(q, k, v, o, lse, do)
+    dq2, dk2, dv2 = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.workspace_bytes(1, 4, 2, 384, 128), dtype=torch.uint8, device=cuda_device)
+    stream = torch.cuda.current_stream().cuda_stream
+    ptr = lambda t: t.data_ptr()
+    rc = fa.bwd_phases_raw(ptr(q), ptr(k), ptr(v), ptr(o), ptr(lse), ptr(do), ptr(dq2), ptr(dk2), ptr(dv2), ptr(ws),
+                           1, 4, 2, 384, 128, True, w.scale, stream)
+    assert rc == 0 and fa.get_status() == 0
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    assert rel_fro(dq2.float().cpu().numpy(), dq1.float().cpu().numpy()) < 1e-3
