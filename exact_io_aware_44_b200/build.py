@@ -1,6 +1,6 @@
 """Build the CUDA library in-tree: nvcc, sm_100a only.
 
-    python -m exact_io_aware_44_b200.build [-v]
+    python exact_io_aware_44_b200/build.py [-v] [--ptxas]
 
 Compiles every csrc/*.cu for sm_100a (object files in parallel) and links
 libfa_b200.so next to this file. The CUDA runtime is linked statically; the
