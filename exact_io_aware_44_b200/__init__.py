@@ -1,7 +1,7 @@
 """Exact IO-aware attention for NVIDIA B200 (sm_100a): Python binding.
 
 A thin ctypes layer over the C ABI in include/fa.h (libfa_b200.so, built
-in-tree by `python -m exact_io_aware_44_b200.build`). It only marshals
+in-tree by `python exact_io_aware_44_b200/build.py`). It only marshals
 arguments: it checks shapes and dtypes, allocates outputs with torch, and
 passes raw device pointers and the current CUDA stream. Every step of the
 attention path runs in the library's CUDA kernels. There is no CPU fallback:
@@ -38,6 +38,7 @@ SIGNATURES = {
     "fa_bwd_preprocess": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "fa_bwd_main": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_convert": (_I, [_P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_get_status": (_I, [_P]),
     "fa_set_wait_budget_ns": (None, [ctypes.c_uint64]),
     "fa_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
@@ -55,7 +56,7 @@ class FAError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_44_b200.build` "
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python exact_io_aware_44_b200/build.py` "
                           "(there is no CPU fallback)")
     so = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():

@@ -324,3 +324,52 @@ int fa_selftest_wait_timeout(uint64_t budget_ns, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fa_bwd_noalloc: the backward pass without a caller-provided workspace, for
+// callers that cannot allocate device memory (see include/fa.h).
+// ---------------------------------------------------------------------------
+namespace fa {
+namespace {
+
+// D and the fp32 dQ accumulator of fa_bwd_noalloc. In host code this name is
+// only a stand-in for the device array: the kernels get its device address,
+// looked up per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+std::mutex g_noalloc_mu;
+
+}  // namespace
+}  // namespace fa
+
+extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                              const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+                              int causal, float scale, void* stream) {
+  bool empty;
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
+  if (rc != FA_OK) return rc;
+  if (fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  DeviceInfo* di;
+  if ((rc = current_device(&di)) != FA_OK) return rc;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_NO_DEVICE;
+  }
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+      // Once per device, with that device current.
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || addr == nullptr) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+      }
+      g_noalloc_addr[dev] = addr;
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  return run_bwd(kPhaseAll, q, k, v, o, lse, dout, dq, dk, dv, scratch, B, Hq, Hkv, N, d, causal, scale, stream);
+}

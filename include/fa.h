@@ -135,6 +135,35 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, c
 int fa_bwd_convert(void* dq, const void* workspace, int B, int Hq, int Hkv, int N, int d, float scale, void* stream);
 
 /*
+ * fa_bwd_noalloc -- fa_bwd for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call: it is a property of this
+ * library's interface, not of the attention method. Some callers cannot call
+ * cudaMalloc: plugins whose host application owns every device allocation,
+ * serving loops that must not hit cudaMalloc's implicit synchronisation, and
+ * fixed-budget deployments that size all device memory up front. They cannot
+ * provide fa_bwd's workspace. This variant computes exactly what fa_bwd
+ * computes, with the same arguments except the workspace: its scratch (D and
+ * the fp32 dQ accumulator) lives in a static device array of
+ * FA_NOALLOC_SCRATCH_BYTES that every GPU which loads the library holds until
+ * the process exits. The call itself allocates nothing.
+ *   Limit     fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) must not exceed
+ *             FA_NOALLOC_SCRATCH_BYTES (about B*Hq*N*(d+1)*4 bytes); larger
+ *             problems return FA_ERR_UNSUPPORTED and launch nothing.
+ *   First use The first call on each device looks up the array's device address
+ *             (which loads the library's kernels on that device). Make that
+ *             first call before any stream capture.
+ *   Sharing   All calls on a device share the one array, which keeps the last
+ *             call's contents; each call re-initialises what it reads. Calls
+ *             whose work overlaps on the GPU (e.g. on two streams) race on it
+ *             and give wrong results: serialise them.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (64ull << 20)
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                   void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                   void* stream);
+
+/*
  * fa_get_status -- synchronise `stream`, then return and clear the device
  * status word of the current device (FA_OK or the first device-side error
  * since the last call). Returns FA_ERR_LAUNCH if the stream reports a CUDA error.
