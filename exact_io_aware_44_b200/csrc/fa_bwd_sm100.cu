@@ -50,12 +50,13 @@ namespace {
 
 constexpr int kBwdThreads = 512;
 // Register split: the launch gives 128 per thread (512 x 128 = 65536). The
-// control warpgroup lowers to 56, the two P/dS warpgroups raise to 160, and
-// the dQ warpgroup keeps the launch count: 128 x (56 + 2 x 160 + 128) = 64512.
+// control and dQ warpgroups lower to 96 and the two P/dS warpgroups raise to
+// 160: 128 x (96 + 2 x 160 + 96) = 65536.
 constexpr int kBwdRegsLaunch = 128;
-constexpr int kBwdRegsControl = 56;
+constexpr int kBwdRegsControl = 96;
 constexpr int kBwdRegsSoftmax = 160;
-static_assert(128 * (kBwdRegsControl + 2 * kBwdRegsSoftmax + kBwdRegsLaunch) <= kBwdThreads * kBwdRegsLaunch,
+constexpr int kBwdRegsDq = 96;
+static_assert(128 * (kBwdRegsControl + 2 * kBwdRegsSoftmax + kBwdRegsDq) <= kBwdThreads * kBwdRegsLaunch,
               "register split");
 
 template <int D>
@@ -281,97 +282,104 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs this role (warp-uniform descriptors, built once and
+    // advanced by constant offsets); lane 0 alone issues tcgen05.mma / commit.
     regs_dec<kBwdRegsControl, kBwdRegsLaunch>();
-    if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16_f32(128, BR, false, false);   // S^T, dP^T
-      constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, false, true);    // dV, dK
-      constexpr uint32_t kIdQ = idesc_bf16_f32(128, 64, true, true);     // dQ (or dQ^T)
-      const uint32_t k_base = smem_u32(smem + C::kOffK);
-      const uint32_t v_base = smem_u32(smem + C::kOffV);
-      const uint32_t st_base = smem_u32(smem + C::kOffStage);
-      const uint32_t pt_base = smem_u32(smem + C::kOffP);
-      const uint32_t ds_base = smem_u32(smem + C::kOffDS);
-      // X^T = A B^T over the head dim: A = K or V tile, B = Q or dO tile (both K-major)
-      auto mma_scores = [&](uint32_t a_base, uint32_t b_base, uint32_t col) {
+    const bool leader = lane == 0;
+    constexpr uint32_t kIdS = idesc_bf16_f32(128, BR, false, false);   // S^T, dP^T
+    constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, false, true);    // dV, dK
+    constexpr uint32_t kIdQ = idesc_bf16_f32(128, 64, true, true);     // dQ (or dQ^T)
+    const uint32_t k_addr = smem_u32(smem + C::kOffK);
+    const uint32_t v_addr = smem_u32(smem + C::kOffV);
+    const uint32_t st_addr = smem_u32(smem + C::kOffStage);
+    const uint32_t pt_addr = smem_u32(smem + C::kOffP);
+    const uint32_t ds_addr = smem_u32(smem + C::kOffDS);
+    // K-major views (LBO unused) and MN-major views (LBO = distance of 64-column blocks)
+    const uint64_t dK_k = sdesc_sw128(k_addr, 16, 1024), dV_k = sdesc_sw128(v_addr, 16, 1024);
+    const uint64_t dSt_k = sdesc_sw128(st_addr, 16, 1024);
+    const uint64_t dSt_mn = sdesc_sw128(st_addr, C::kQRegion, 1024);
+    const uint64_t dPt_k = sdesc_sw128(pt_addr, 16, 1024), dDs_k = sdesc_sw128(ds_addr, 16, 1024);
+    const uint64_t dK_mn = sdesc_sw128(k_addr, C::kKVRegion, 1024);
+    const uint64_t dDs_mn = sdesc_sw128(ds_addr, C::kPRegion, 1024);
+    // X^T = A B^T over the head dim: A = K or V tile, B = Q or dO tile (both K-major)
+    auto mma_scores = [&](uint64_t a0, uint64_t b0, uint32_t col) {
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t a = sdesc_sw128(a_base + (k >> 2) * C::kKVRegion + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b_base + (k >> 2) * C::kQRegion + (k & 3) * 32, 16, 1024);
-          mma_bf16_ss(tmem + col, a, bd, kIdS, k > 0 ? 1u : 0u);
-        }
-      };
-      // acc += A B over the query rows: A = P^T or dS^T (K-major), B = dO or Q (MN-major)
-      auto mma_accum = [&](uint32_t a_base, uint32_t b_base, uint32_t col, bool first) {
-#pragma unroll
-        for (int k = 0; k < BR / 16; ++k) {
-          const uint64_t a = sdesc_sw128(a_base + (k >> 2) * C::kPRegion + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b_base + k * 2048, C::kQRegion, 1024);
-          mma_bf16_ss(tmem + col, a, bd, kIdKV, (!first || k > 0) ? 1u : 0u);
-        }
-      };
-      // dQ (d = 64): A = dS (MN-major view of dS^T), B = K (MN-major), over the 128 keys.
-      // dQ^T (d = 128): A = K^T (MN-major view of K), B = dS^T (MN-major), over the 128 keys.
-      auto mma_dq = [&]() {
-#pragma unroll
-        for (int k = 0; k < kTileN / 16; ++k) {
-          uint64_t a, bd;
-          if (D == 128) {
-            a = sdesc_sw128(k_base + k * 2048, C::kKVRegion, 1024);
-            bd = sdesc_sw128(ds_base + k * 2048, C::kPRegion, 1024);
-          } else {
-            a = sdesc_sw128(ds_base + k * 2048, C::kPRegion, 1024);
-            bd = sdesc_sw128(k_base + k * 2048, C::kKVRegion, 1024);
-          }
-          mma_bf16_ss(tmem + C::kColDQ, a, bd, kIdQ, k > 0 ? 1u : 0u);
-        }
-      };
-      auto stage_addr = [&](int it) { return st_base + (it % ST) * C::kStageBytes; };
-      bool ok = mbar_wait(kv_full, 0, w);
-      if (ok && n_it > 0) ok = mbar_wait(&st_full[0], 0, w);
-      tc_fence_after();
-      if (ok && n_it > 0) {
-        mma_scores(k_base, stage_addr(0), C::kColS);
-        mma_commit(s_full);
-        mma_scores(v_base, stage_addr(0) + C::kQBytes, C::kColDP);
-        mma_commit(dp_full);
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t ao = (k >> 2) * C::kKVRegion + (k & 3) * 32;
+        const uint32_t bo = (k >> 2) * C::kQRegion + (k & 3) * 32;
+        if (leader) mma_bf16_ss(tmem + col, desc_advance(a0, ao), desc_advance(b0, bo), kIdS, k > 0 ? 1u : 0u);
       }
-      for (int it = 0; it < n_it && ok; ++it) {
-        const uint32_t sa = stage_addr(it);
-        const uint32_t ph = it & 1;
-        // dV += P^T dO_i
-        if (!(ok = mbar_wait(p_full, ph, w))) break;
+    };
+    // acc += A B over the query rows: A = P^T or dS^T (K-major), B = dO or Q (MN-major)
+    auto mma_accum = [&](uint64_t a0, uint64_t b0, uint32_t col, bool first) {
+#pragma unroll
+      for (int k = 0; k < BR / 16; ++k) {
+        const uint32_t ao = (k >> 2) * C::kPRegion + (k & 3) * 32;
+        if (leader)
+          mma_bf16_ss(tmem + col, desc_advance(a0, ao), desc_advance(b0, k * 2048), kIdKV,
+                      (!first || k > 0) ? 1u : 0u);
+      }
+    };
+    // dQ (d = 64): A = dS (MN-major view of dS^T), B = K (MN-major), over the 128 keys.
+    // dQ^T (d = 128): A = K^T (MN-major view of K), B = dS^T (MN-major), over the 128 keys.
+    auto mma_dq = [&]() {
+      const uint64_t a0 = (D == 128) ? dK_mn : dDs_mn;
+      const uint64_t b0 = (D == 128) ? dDs_mn : dK_mn;
+#pragma unroll
+      for (int k = 0; k < kTileN / 16; ++k)
+        if (leader) mma_bf16_ss(tmem + C::kColDQ, desc_advance(a0, k * 2048), desc_advance(b0, k * 2048), kIdQ,
+                                k > 0 ? 1u : 0u);
+    };
+    auto stage_off = [&](int it) -> uint32_t { return (uint32_t)((it % ST) * C::kStageBytes); };
+    bool ok = mbar_wait(kv_full, 0, w);
+    if (ok && n_it > 0) ok = mbar_wait(&st_full[0], 0, w);
+    tc_fence_after();
+    if (ok && n_it > 0) {
+      mma_scores(dK_k, dSt_k, C::kColS);
+      if (leader) mma_commit(s_full);
+      mma_scores(dV_k, desc_advance(dSt_k, C::kQBytes), C::kColDP);
+      if (leader) mma_commit(dp_full);
+    }
+    for (int it = 0; it < n_it && ok; ++it) {
+      const uint32_t so = stage_off(it);
+      const uint32_t ph = it & 1;
+      // dV += P^T dO_i
+      if (!(ok = mbar_wait(p_full, ph, w))) break;
+      tc_fence_after();
+      mma_accum(dPt_k, desc_advance(dSt_mn, so + C::kQBytes), C::kColDV, it == 0);
+      if (leader) mma_commit(p_free);
+      // the next tile's S^T and dP^T, as soon as their TMEM buffers were read
+      if (it + 1 < n_it) {
+        const uint32_t so1 = stage_off(it + 1);
+        if (!(ok = mbar_wait(&st_full[(it + 1) % ST], ((it + 1) / ST) & 1, w))) break;
+        if (!(ok = mbar_wait(s_free, ph, w))) break;
         tc_fence_after();
-        mma_accum(pt_base, sa + C::kQBytes, C::kColDV, it == 0);
-        mma_commit(p_free);
-        // the next tile's S^T and dP^T, as soon as their TMEM buffers were read
-        if (it + 1 < n_it) {
-          if (!(ok = mbar_wait(&st_full[(it + 1) % ST], ((it + 1) / ST) & 1, w))) break;
-          if (!(ok = mbar_wait(s_free, ph, w))) break;
-          tc_fence_after();
-          mma_scores(k_base, stage_addr(it + 1), C::kColS);
-          mma_commit(s_full);
-          if (!(ok = mbar_wait(dp_free, ph, w))) break;
-          tc_fence_after();
-          mma_scores(v_base, stage_addr(it + 1) + C::kQBytes, C::kColDP);
-          mma_commit(dp_full);
-        }
-        // dK += dS^T Q_i ; dQ_i
-        if (!(ok = mbar_wait(ds_full, ph, w))) break;
+        mma_scores(dK_k, desc_advance(dSt_k, so1), C::kColS);
+        if (leader) mma_commit(s_full);
+        if (!(ok = mbar_wait(dp_free, ph, w))) break;
         tc_fence_after();
-        mma_accum(ds_base, sa, C::kColDK, it == 0);
-        if (it >= 1 && !(ok = mbar_wait(dq_free, ph ^ 1, w))) break;
-        tc_fence_after();
-        mma_dq();
+        mma_scores(dV_k, desc_advance(dSt_k, so1 + C::kQBytes), C::kColDP);
+        if (leader) mma_commit(dp_full);
+      }
+      // dK += dS^T Q_i ; dQ_i
+      if (!(ok = mbar_wait(ds_full, ph, w))) break;
+      tc_fence_after();
+      mma_accum(dDs_k, desc_advance(dSt_mn, so), C::kColDK, it == 0);
+      if (it >= 1 && !(ok = mbar_wait(dq_free, ph ^ 1, w))) break;
+      tc_fence_after();
+      mma_dq();
+      if (leader) {
         mma_commit(dq_full);
         mma_commit(ds_free);
         mma_commit(&st_empty[it % ST]);
       }
-      mma_commit(mma_done);
-      WaitCtx drain{abort_flag, p.status, 20000000ull};
-      volatile int zero = 0;
-      drain.abort_flag = &zero;
-      mbar_wait(mma_done, 0, drain);
     }
+    if (leader) mma_commit(mma_done);
+    __syncwarp();
+    WaitCtx drain{abort_flag, p.status, 20000000ull};
+    volatile int zero = 0;
+    drain.abort_flag = &zero;
+    mbar_wait(mma_done, 0, drain);
   } else if (warp < 4) {
     regs_dec<kBwdRegsControl, kBwdRegsLaunch>();
   } else if (warp < 12) {
@@ -458,6 +466,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ reductions, dK / dV epilogue
+    regs_dec<kBwdRegsDq, kBwdRegsLaunch>();
     const int quarter = warp & 3;
     const int tl = quarter * 32 + lane;  // TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;

@@ -27,8 +27,9 @@
 //
 // The MMA issue order per key tile j is S_0(j), S_1(j), PV_0(j-1), PV_1(j-1),
 // so the tensor core computes the next scores while both softmax warpgroups
-// exponentiate the current ones. The shared-memory ring holds tiles in the
-// same order: K_0, K_1, V_0, K_2, V_1, ..., V_last.
+// exponentiate the current ones. K and V tiles stream through two separate
+// rings of shared-memory stages, so loading K_{j+1} only waits for the scores
+// of K_{j-1} (not for the P V products of V_{j-1}).
 #include <math.h>
 
 #include "fa_internal.h"
@@ -38,17 +39,19 @@ namespace fa {
 namespace {
 
 constexpr int kFwdThreads = 384;
-// Register split: 384 threads x 168 at launch = 64512 = 128 x 56 (producer /
-// MMA warpgroup) + 256 x 224 (the two softmax warpgroups).
+// Register split: 384 threads x 168 at launch = 64512 = 128 x 88 (producer /
+// MMA warpgroup) + 256 x 208 (the two softmax warpgroups).
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsControl = 56;
-constexpr int kRegsSoftmax = 224;
+constexpr int kRegsControl = 88;
+constexpr int kRegsSoftmax = 208;
 static_assert(kFwdThreads * kRegsLaunch == 128 * kRegsControl + 256 * kRegsSoftmax, "register split");
 constexpr uint32_t kRescaleThresholdLog2 = 8;  // rescale only when m grows by > 2^8
 
 template <int D>
 struct FwdCfg {
-  static constexpr int kStages = (D == 128) ? 3 : 6;
+  static constexpr int kStagesK = (D == 128) ? 2 : 3;  // K ring
+  static constexpr int kStagesV = (D == 128) ? 1 : 3;  // V ring
+  static constexpr int kStages = kStagesK + kStagesV;
   static constexpr int kTileBytes = kTileM * D * 2;      // one Q, K or V tile (bf16)
   static constexpr int kPBytes = kTileM * kTileN * 2;    // one P tile (bf16)
   static constexpr int kRegion = kTileM * 128;           // one 64-column block of a tile
@@ -56,7 +59,8 @@ struct FwdCfg {
   static constexpr int kOffP = kOffQ + 2 * kTileBytes;
   static constexpr int kOffKV = kOffP + 2 * kPBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  // q_full, ring_full[S], ring_empty[S], s_ready[2], s_free[2], p_ready[2], pv_done[2], mma_final
+  // q_full, full[S], empty[S] (K ring slots first, then V ring), s_ready[2], s_free[2],
+  // p_ready[2], pv_done[2], mma_final
   static constexpr int kNumBars = 1 + 2 * kStages + 9;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
@@ -147,107 +151,123 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int z = 0; z < D / 64; ++z)
           tma_load_3d(smem + C::kOffQ + t * C::kTileBytes + z * C::kRegion, &tmQ, q_full, z * 64,
                       q0 + t * kTileM, q_head);
-      int it = 0;
-      auto push = [&](const CUtensorMap* map, int kv_tile) -> bool {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
+      // ring r (0 = K, 1 = V): slots [base[r], base[r] + n[r]), cnt[r] tiles pushed so far
+      const int base[2] = {0, C::kStagesK};
+      const int nst[2] = {C::kStagesK, C::kStagesV};
+      int cnt[2] = {0, 0};
+      auto push = [&](int r, int kv_tile) -> bool {
+        const int s = base[r] + cnt[r] % nst[r];
+        const uint32_t ph = (cnt[r] / nst[r]) & 1;
         if (!mbar_wait(&ring_empty[s], ph ^ 1, w)) return false;
         mbar_arrive_expect_tx(&ring_full[s], C::kTileBytes);
+        const CUtensorMap* map = r == 0 ? &tmK : &tmV;
 #pragma unroll
         for (int z = 0; z < D / 64; ++z)
           tma_load_3d(smem + C::kOffKV + s * C::kTileBytes + z * C::kRegion, map, &ring_full[s], z * 64,
                       kv_tile * kTileN, kv_head);
-        ++it;
+        ++cnt[r];
         return true;
       };
       bool ok = true;
       for (int j = 0; j < n_kv && ok; ++j) {
-        ok = push(&tmK, j);
-        if (ok && j >= 1) ok = push(&tmV, j - 1);
+        ok = push(0, j);
+        if (ok && j >= 1) ok = push(1, j - 1);
       }
-      if (ok) ok = push(&tmV, n_kv - 1);
+      if (ok) ok = push(1, n_kv - 1);
       if (!ok) {
         // Error path: let the loads already issued land before the CTA exits.
         WaitCtx drain{abort_flag, p.status, 20000000ull};
         volatile int zero = 0;
         drain.abort_flag = &zero;
-        for (int k = max(0, it - S); k < it; ++k) mbar_wait(&ring_full[k % S], (k / S) & 1, drain);
+        for (int r = 0; r < 2; ++r)
+          for (int k = max(0, cnt[r] - nst[r]); k < cnt[r]; ++k)
+            mbar_wait(&ring_full[base[r] + k % nst[r]], (k / nst[r]) & 1, drain);
         mbar_wait(q_full, 0, drain);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs this role so that descriptors are warp-uniform; lane 0
+    // alone issues tcgen05.mma and tcgen05.commit. Descriptors are built once
+    // and advanced by constant offsets of the start-address field: recomputing
+    // them per MMA from runtime indices halves the issue rate.
     regs_dec<kRegsControl, kRegsLaunch>();
-    if (lane == 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
-      constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, false, true);
-      const uint32_t q_base = smem_u32(smem + C::kOffQ);
-      const uint32_t p_base = smem_u32(smem + C::kOffP);
-      const uint32_t kv_base = smem_u32(smem + C::kOffKV);
-      int it = 0;
-      bool ok = mbar_wait(q_full, 0, w);
+    const bool leader = lane == 0;
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, false, true);
+    const uint64_t d_q = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+    const uint64_t d_p = sdesc_sw128(smem_u32(smem + C::kOffP), 16, 1024);
+    const uint64_t d_k = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);           // K-major view
+    const uint64_t d_v = sdesc_sw128(smem_u32(smem + C::kOffKV), C::kRegion, 1024);   // MN-major view
+    const int base[2] = {0, C::kStagesK};
+    const int nst[2] = {C::kStagesK, C::kStagesV};
+    int cnt[2] = {0, 0};
+    bool ok = mbar_wait(q_full, 0, w);
+    tc_fence_after();
+    auto take = [&](int r, int& slot) -> bool {  // next tile of ring r (0 = K, 1 = V)
+      slot = base[r] + cnt[r] % nst[r];
+      const bool res = mbar_wait(&ring_full[slot], (cnt[r] / nst[r]) & 1, w);
+      ++cnt[r];
       tc_fence_after();
-      auto take = [&](int& slot) -> bool {
-        slot = it % S;
-        const bool r = mbar_wait(&ring_full[slot], (it / S) & 1, w);
-        ++it;
-        tc_fence_after();
-        return r;
-      };
-      auto issue_s = [&](int t, int slot) {
+      return res;
+    };
+    auto issue_s = [&](int t, int slot) {
+      const uint64_t a0 = desc_advance(d_q, t * C::kTileBytes);
+      const uint64_t b0 = desc_advance(d_k, slot * C::kTileBytes);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * C::kRegion + (k & 3) * 32;
-          const uint64_t a = sdesc_sw128(q_base + t * C::kTileBytes + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(kv_base + slot * C::kTileBytes + off, 16, 1024);
-          mma_bf16_ss(tmem + t * 128, a, bd, kIdescS, k > 0 ? 1u : 0u);
-        }
-        mma_commit(&s_ready[t]);
-      };
-      auto issue_pv = [&](int t, int slot, int j) {
-#pragma unroll
-        for (int k = 0; k < kTileN / 16; ++k) {
-          const uint64_t a = sdesc_sw128(p_base + t * C::kPBytes + (k >> 2) * C::kRegion + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(kv_base + slot * C::kTileBytes + k * 16 * 128, C::kRegion, 1024);
-          mma_bf16_ss(tmem + 256 + t * 128, a, bd, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
-        }
-        mma_commit(&pv_done[t]);
-      };
-      auto do_pv = [&](int j) -> bool {  // PV_0(j), PV_1(j) from the V_j stage
-        int slot;
-        if (!take(slot)) return false;
-        for (int t = 0; t < 2; ++t) {
-          if (j >= n_iter[t]) continue;
-          if (!mbar_wait(&p_ready[t], j & 1, w)) return false;
-          tc_fence_after();
-          issue_pv(t, slot, j);
-        }
-        mma_commit(&ring_empty[slot]);
-        return true;
-      };
-      for (int j = 0; j < n_kv && ok; ++j) {
-        int slot;
-        ok = take(slot);
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= n_iter[t]) continue;
-          if (j > 0) {
-            ok = mbar_wait(&s_free[t], (j - 1) & 1, w);
-            tc_fence_after();
-          }
-          if (ok) issue_s(t, slot);
-        }
-        if (!ok) break;
-        mma_commit(&ring_empty[slot]);
-        if (j >= 1) ok = do_pv(j - 1);
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * C::kRegion + (k & 3) * 32;
+        if (leader) mma_bf16_ss(tmem + t * 128, desc_advance(a0, off), desc_advance(b0, off), kIdescS, k > 0 ? 1u : 0u);
       }
-      if (ok) ok = do_pv(n_kv - 1);
-      // Every MMA issued above must finish before TMEM is released.
-      mma_commit(mma_final);
-      WaitCtx drain{abort_flag, p.status, 20000000ull};
-      volatile int zero = 0;
-      drain.abort_flag = &zero;
-      mbar_wait(mma_final, 0, drain);
+      if (leader) mma_commit(&s_ready[t]);
+    };
+    auto issue_pv = [&](int t, int slot, int j) {
+      const uint64_t a0 = desc_advance(d_p, t * C::kPBytes);
+      const uint64_t b0 = desc_advance(d_v, slot * C::kTileBytes);
+#pragma unroll
+      for (int k = 0; k < kTileN / 16; ++k) {
+        const uint32_t aoff = (k >> 2) * C::kRegion + (k & 3) * 32;
+        if (leader)
+          mma_bf16_ss(tmem + 256 + t * 128, desc_advance(a0, aoff), desc_advance(b0, k * 16 * 128), kIdescPV,
+                      (j > 0 || k > 0) ? 1u : 0u);
+      }
+      if (leader) mma_commit(&pv_done[t]);
+    };
+    auto do_pv = [&](int j) -> bool {  // PV_0(j), PV_1(j) from the V_j stage
+      int slot;
+      if (!take(1, slot)) return false;
+      for (int t = 0; t < 2; ++t) {
+        if (j >= n_iter[t]) continue;
+        if (!mbar_wait(&p_ready[t], j & 1, w)) return false;
+        tc_fence_after();
+        issue_pv(t, slot, j);
+      }
+      if (leader) mma_commit(&ring_empty[slot]);
+      return true;
+    };
+    for (int j = 0; j < n_kv && ok; ++j) {
+      int slot;
+      ok = take(0, slot);
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (j >= n_iter[t]) continue;
+        if (j > 0) {
+          ok = mbar_wait(&s_free[t], (j - 1) & 1, w);
+          tc_fence_after();
+        }
+        if (ok) issue_s(t, slot);
+      }
+      if (!ok) break;
+      if (leader) mma_commit(&ring_empty[slot]);
+      if (j >= 1) ok = do_pv(j - 1);
     }
+    if (ok) ok = do_pv(n_kv - 1);
+    // Every MMA issued above must finish before TMEM is released.
+    if (leader) mma_commit(mma_final);
+    __syncwarp();
+    WaitCtx drain{abort_flag, p.status, 20000000ull};
+    volatile int zero = 0;
+    drain.abort_flag = &zero;
+    mbar_wait(mma_final, 0, drain);
   } else if (warp < 4) {
     regs_dec<kRegsControl, kRegsLaunch>();
   } else {
@@ -294,9 +314,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int i = 0; i < kTileN; ++i)
             if (i >= lim) s[i] = -INFINITY;
         }
-        float mx = s[0];
+        // row max: four independent chains of 3-input max
+        float mq[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-        for (int i = 1; i < kTileN; ++i) mx = fmaxf(mx, s[i]);
+        for (int i = 4; i < kTileN; i += 8) {
+          mq[0] = fmax3(mq[0], s[i], s[i + 1]);
+          mq[1] = fmax3(mq[1], s[i + 2], s[i + 3]);
+          mq[2] = fmax3(mq[2], s[i + 4], s[i + 5]);
+          if (i + 6 < kTileN) mq[3] = fmax3(mq[3], s[i + 6], s[i + 7]);
+        }
+        const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
         const float m_new = fmaxf(m_ref, mx);
         float alpha = 1.f;
         bool rescale = false;
@@ -311,15 +338,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
         // P = 2^(S c - m c), packed to bf16 pairs at once; l sums the fp32 values.
         uint32_t pk[kTileN / 2];
-        float rs = 0.f;
+        uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int i = 0; i < kTileN; i += 2) {
           const float e0 = ex2(fmaf(s[i], c, -mc));
           const float e1 = ex2(fmaf(s[i + 1], c, -mc));
-          rs += e0 + e1;
+          rs2[(i >> 1) & 1] = f2_add(rs2[(i >> 1) & 1], f2_pack(e0, e1));
           pk[i / 2] = pack_bf16x2(e0, e1);
         }
-        l += rs;
+        float ra, rb, rc, rd;
+        f2_unpack(rs2[0], ra, rb);
+        f2_unpack(rs2[1], rc, rd);
+        l += (ra + rb) + (rc + rd);
 
         if (j >= 1) {
           // PV(j-1) must be done: it reads the P buffer and accumulates into O.
