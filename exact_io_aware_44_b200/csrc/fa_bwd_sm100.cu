@@ -22,7 +22,7 @@
 //
 // bwd_main roles (512 threads):
 //   warp 0      producer: K, V once (TMA); per query tile Q_i, dO_i (TMA) and
-//               LSE_i log2(e), D_i (plain loads) into a ring of stages.
+//               -LSE_i log2(e), D_i (plain loads) into a ring of stages.
 //   warp 1      allocates TMEM; one lane issues every tcgen05.mma.
 //   warps 4-11  two warpgroups, thread = key row; warpgroup h computes P^T and
 //               dS^T for query columns [h BR/2, (h+1) BR/2) and writes them to
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int r = lane; r < BR; r += 32) {
         const int i = i0 + r;
         const bool in = i < p.N;
-        lse2[r] = in ? p.lse[rbase + i] * 1.4426950408889634f : INFINITY;
+        lse2[r] = in ? -p.lse[rbase + i] * 1.4426950408889634f : -INFINITY;  // -LSE log2(e)
         dl[r] = in ? p.delta[rbase + i] : 0.f;
       }
       mbar_arrive(&st_full[s]);
@@ -416,13 +416,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(s_free);
-      // P^T[key][q] = 2^(S c - LSE2_q), zero for future queries and invalid keys.
-      const bool diag = p.causal && i0 < j0 + kTileN;
+      // P^T[key][q] = 2^(S c - LSE_q log2 e), zero for future queries and invalid keys.
+      // The stage holds -LSE log2(e) per query (-inf past N), read as broadcast pairs.
+      const uint64_t c2 = f2_pack(c, c);
+      const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2);
 #pragma unroll
-      for (int i = 0; i < HB; ++i) {
-        float e = ex2(fmaf(pr[i], c, -lse2[i]));
-        if (diag && i0 + i < key) e = 0.f;
-        pr[i] = key_valid ? e : 0.f;
+      for (int i = 0; i < HB; i += 2) {
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(pr[i], pr[i + 1]), c2, nl2[i / 2]), x0, x1);
+        pr[i] = ex2(x0);
+        pr[i + 1] = ex2(x1);
+      }
+      if (p.causal && i0 < j0 + kTileN) {  // diagonal tiles only
+#pragma unroll
+        for (int i = 0; i < HB; ++i)
+          if (i0 + i < key) pr[i] = 0.f;
+      }
+      if (!key_valid) {
+#pragma unroll
+        for (int i = 0; i < HB; ++i) pr[i] = 0.f;
       }
       if (it >= 1 && !mbar_wait(p_free, ph ^ 1, w)) break;
 #pragma unroll
@@ -451,9 +463,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       mbar_arrive(dp_free);
       uint32_t dsp[HB / 2];
+      const uint64_t* dl2 = reinterpret_cast<const uint64_t*>(dl);
 #pragma unroll
-      for (int i = 0; i < HB; i += 2)
-        dsp[i / 2] = pack_bf16x2(pr[i] * (dp[i] - dl[i]), pr[i + 1] * (dp[i + 1] - dl[i + 1]));
+      for (int i = 0; i < HB; i += 2) {
+        float a, bb;
+        f2_unpack(f2_mul(f2_pack(pr[i], pr[i + 1]), f2_sub(f2_pack(dp[i], dp[i + 1]), dl2[i / 2])), a, bb);
+        dsp[i / 2] = pack_bf16x2(a, bb);
+      }
       if (it >= 1 && !mbar_wait(ds_free, ph ^ 1, w)) break;
 #pragma unroll
       for (int ch = 0; ch < HB / 8; ++ch) {
