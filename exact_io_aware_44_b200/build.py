@@ -56,6 +56,7 @@ def build(verbose: bool = False, ptxas_info: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     extra = ["-Xptxas", "-v"] if ptxas_info else []
+    extra += os.environ.get("FA_NVCC_EXTRA", "").split()  # e.g. -DFA_CONSUMER_POLL_NS=100
     with cf.ThreadPoolExecutor(max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose or ptxas_info, extra), srcs))
     newest = max(os.path.getmtime(o) for o in objs)

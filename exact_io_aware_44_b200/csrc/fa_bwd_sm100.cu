@@ -30,9 +30,10 @@
 //   warps 12-15 thread = TMEM lane of the dQ tile: reads it and issues the fp32
 //               reductions; at the end, writes dK and dV.
 //
-// MMA issue order per query tile i: dV(i), S(i+1), dP(i+1), dK(i), dQ(i). The
-// next tile's scores and dP are computed while the elementwise warpgroups
-// still work on dS(i) and P(i+1), so the tensor core always has queued work.
+// MMA issue order per query tile i: S(i+1), dV(i), dP(i+1), dK(i), dQ(i). The
+// next tile's scores are issued as soon as the current ones have been read out
+// of TMEM, and dP(i+1) as soon as dP(i) has, so they are computed while the
+// elementwise warpgroups still work on P(i) and dS(i).
 //
 // Query tiles are BR = 64 rows for d = 128 (so dQ^T = K^T dS^T has M = d = 128)
 // and BR = 128 rows for d = 64 (so dQ = dS K has M = 128 query rows). TMEM
@@ -257,7 +258,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int h = kvh * g + it / per_head;
       const int i0 = (qt_first + it % per_head) * BR;
       const int q_head = b * p.Hq + h;
-      ok = mbar_wait(&st_empty[s], ((it / ST) & 1) ^ 1, w);
+      ok = mbar_wait_spin(&st_empty[s], ((it / ST) & 1) ^ 1, w);
       if (!ok) break;
       uint8_t* stage = smem + C::kOffStage + s * C::kStageBytes;
       if (lane == 0) {
@@ -331,8 +332,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                 k > 0 ? 1u : 0u);
     };
     auto stage_off = [&](int it) -> uint32_t { return (uint32_t)((it % ST) * C::kStageBytes); };
-    bool ok = mbar_wait(kv_full, 0, w);
-    if (ok && n_it > 0) ok = mbar_wait(&st_full[0], 0, w);
+    bool ok = mbar_wait_spin(kv_full, 0, w);
+    if (ok && n_it > 0) ok = mbar_wait_spin(&st_full[0], 0, w);
     tc_fence_after();
     if (ok && n_it > 0) {
       mma_scores(dK_k, dSt_k, C::kColS);
@@ -343,29 +344,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int it = 0; it < n_it && ok; ++it) {
       const uint32_t so = stage_off(it);
       const uint32_t ph = it & 1;
+      // the next tile's S^T as soon as the current one has been read out of TMEM
+      if (it + 1 < n_it) {
+        if (!(ok = mbar_wait_spin(&st_full[(it + 1) % ST], ((it + 1) / ST) & 1, w))) break;
+        if (!(ok = mbar_wait_spin(s_free, ph, w))) break;
+        tc_fence_after();
+        mma_scores(dK_k, desc_advance(dSt_k, stage_off(it + 1)), C::kColS);
+        if (leader) mma_commit(s_full);
+      }
       // dV += P^T dO_i
-      if (!(ok = mbar_wait(p_full, ph, w))) break;
+      if (!(ok = mbar_wait_spin(p_full, ph, w))) break;
       tc_fence_after();
       mma_accum(dPt_k, desc_advance(dSt_mn, so + C::kQBytes), C::kColDV, it == 0);
       if (leader) mma_commit(p_free);
-      // the next tile's S^T and dP^T, as soon as their TMEM buffers were read
+      // the next tile's dP^T once the current one has been read out
       if (it + 1 < n_it) {
-        const uint32_t so1 = stage_off(it + 1);
-        if (!(ok = mbar_wait(&st_full[(it + 1) % ST], ((it + 1) / ST) & 1, w))) break;
-        if (!(ok = mbar_wait(s_free, ph, w))) break;
+        if (!(ok = mbar_wait_spin(dp_free, ph, w))) break;
         tc_fence_after();
-        mma_scores(dK_k, desc_advance(dSt_k, so1), C::kColS);
-        if (leader) mma_commit(s_full);
-        if (!(ok = mbar_wait(dp_free, ph, w))) break;
-        tc_fence_after();
-        mma_scores(dV_k, desc_advance(dSt_k, so1 + C::kQBytes), C::kColDP);
+        mma_scores(dV_k, desc_advance(dSt_k, stage_off(it + 1) + C::kQBytes), C::kColDP);
         if (leader) mma_commit(dp_full);
       }
       // dK += dS^T Q_i ; dQ_i
-      if (!(ok = mbar_wait(ds_full, ph, w))) break;
+      if (!(ok = mbar_wait_spin(ds_full, ph, w))) break;
       tc_fence_after();
       mma_accum(dDs_k, desc_advance(dSt_mn, so), C::kColDK, it == 0);
-      if (it >= 1 && !(ok = mbar_wait(dq_free, ph ^ 1, w))) break;
+      if (it >= 1 && !(ok = mbar_wait_spin(dq_free, ph ^ 1, w))) break;
       tc_fence_after();
       mma_dq();
       if (leader) {
@@ -402,8 +405,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* lse2 =
           reinterpret_cast<const float*>(smem + C::kOffStage + s * C::kStageBytes + 2 * C::kQBytes) + col0;
       const float* dl = lse2 + BR;
-      if (!mbar_wait(&st_full[s], (it / ST) & 1, w)) break;
-      if (!mbar_wait(s_full, ph, w)) break;
+      if (!mbar_wait_ns(&st_full[s], (it / ST) & 1, w, kConsumerPollNs)) break;
+      if (!mbar_wait_ns(s_full, ph, w, kConsumerPollNs)) break;
       tc_fence_after();
       float pr[HB];
 #pragma unroll
@@ -436,7 +439,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int i = 0; i < HB; ++i) pr[i] = 0.f;
       }
-      if (it >= 1 && !mbar_wait(p_free, ph ^ 1, w)) break;
+      if (it >= 1 && !mbar_wait_ns(p_free, ph ^ 1, w, kConsumerPollNs)) break;
 #pragma unroll
       for (int ch = 0; ch < HB / 8; ++ch) {
         const int c0 = ch * 8;
@@ -449,7 +452,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(p_full);
       // dS^T = P^T o (dP^T - D_q); dP^T is read out whole first so the next
       // tile's dP^T can be issued at once.
-      if (!mbar_wait(dp_full, ph, w)) break;
+      if (!mbar_wait_ns(dp_full, ph, w, kConsumerPollNs)) break;
       tc_fence_after();
       float dp[HB];
 #pragma unroll
@@ -470,7 +473,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         f2_unpack(f2_mul(f2_pack(pr[i], pr[i + 1]), f2_sub(f2_pack(dp[i], dp[i + 1]), dl2[i / 2])), a, bb);
         dsp[i / 2] = pack_bf16x2(a, bb);
       }
-      if (it >= 1 && !mbar_wait(ds_free, ph ^ 1, w)) break;
+      if (it >= 1 && !mbar_wait_ns(ds_free, ph ^ 1, w, kConsumerPollNs)) break;
 #pragma unroll
       for (int ch = 0; ch < HB / 8; ++ch) {
         const int chunk = col0 / 8 + ch;
@@ -491,7 +494,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int h = kvh * g + it / per_head;
       const int i0 = (qt_first + it % per_head) * BR;
       const size_t head_row0 = (size_t)(b * p.Hq + h) * p.N;
-      if (!(ok = mbar_wait(dq_full, it & 1, w))) break;
+      if (!(ok = mbar_wait_ns(dq_full, it & 1, w, kConsumerPollNs))) break;
       tc_fence_after();
       uint32_t r0[32], r1[32];
       tmem_ld32(tmem + lane_off + C::kColDQ, r0);

@@ -8,28 +8,32 @@
 // matrix only ever exists as one 128 x 128 tile in Tensor Memory.
 //
 // One CTA owns two 128-row query tiles of one (batch, head) and 384 threads:
-//   warp 0      TMA producer: Q once, then K_j / V_j tiles through a ring of
-//               shared-memory stages guarded by mbarriers (full / empty).
-//   warp 1      allocates Tensor Memory; one lane issues every tcgen05.mma:
-//               S_t = Q_t K_j^T into TMEM, then O_t += P_t V_j into TMEM.
+//   warp 0      TMA producer: Q once, then K_0, V_0, K_1, V_1, ... through one
+//               ring of shared-memory stages guarded by mbarriers (full / empty).
+//   warp 1      allocates Tensor Memory; lane 0 issues every tcgen05.mma:
+//               S_t = Q_t K_j^T into TMEM, then O_t += P_t V_j with P_t read
+//               from TMEM.
 //   warps 4-7   softmax for query tile 0 (thread = query row = TMEM lane).
 //   warps 8-11  softmax for query tile 1.
-// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 [384,384+d).
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 [384,384+d);
+// P_t (bf16 pairs, 64 columns) overwrites the first half of S_t once it is read.
 //
 // Per key tile j, a softmax thread loads its row of S_t, applies the causal
 // mask on the diagonal tile, updates the running max, and computes
 // P = 2^(S c - m c) with c = scale * log2(e) on the SFU. It rescales its row
 // of O_t in TMEM only when the max grew by more than 2^8; otherwise the stale
 // max stays the reference, which is exact because the final division uses the
-// same reference. P is written to shared memory as bf16 in the 128-byte-swizzled
-// K-major layout that tcgen05.mma reads. The epilogue divides O by l, stores O
-// as bf16 and writes LSE = (m c + log2 l) ln 2.
+// same reference. It stores P as bf16 into Tensor Memory, where the P V product
+// reads it: P never touches shared memory, whose bandwidth the score MMAs and
+// the K/V loads already use. The epilogue divides O by l, stores O as bf16 and
+// writes LSE = (m c + log2 l) ln 2.
 //
-// The MMA issue order per key tile j is S_0(j), S_1(j), PV_0(j-1), PV_1(j-1),
-// so the tensor core computes the next scores while both softmax warpgroups
-// exponentiate the current ones. K and V tiles stream through two separate
-// rings of shared-memory stages, so loading K_{j+1} only waits for the scores
-// of K_{j-1} (not for the P V products of V_{j-1}).
+// MMA issue order: S_0(0), S_1(0), then per key tile j: PV_0(j), S_0(j+1),
+// PV_1(j), S_1(j+1). S_t(j+1) overwrites the columns PV_t(j) reads; one
+// thread's MMAs execute in issue order. The commit after S_t(j+1) also covers
+// PV_t(j), so when a softmax warpgroup sees S_t(j+1), O_t is complete and may be
+// rescaled. While one softmax warpgroup exponentiates, the tensor core runs the
+// other tile's P V and scores.
 #include <math.h>
 
 #include "fa_internal.h"
@@ -49,19 +53,14 @@ constexpr uint32_t kRescaleThresholdLog2 = 8;  // rescale only when m grows by >
 
 template <int D>
 struct FwdCfg {
-  static constexpr int kStagesK = (D == 128) ? 2 : 3;  // K ring
-  static constexpr int kStagesV = (D == 128) ? 1 : 3;  // V ring
-  static constexpr int kStages = kStagesK + kStagesV;
-  static constexpr int kTileBytes = kTileM * D * 2;      // one Q, K or V tile (bf16)
-  static constexpr int kPBytes = kTileM * kTileN * 2;    // one P tile (bf16)
-  static constexpr int kRegion = kTileM * 128;           // one 64-column block of a tile
+  static constexpr int kStages = (D == 128) ? 5 : 10;  // K/V ring, in order K_0, V_0, K_1, V_1, ...
+  static constexpr int kTileBytes = kTileM * D * 2;    // one Q, K or V tile (bf16)
+  static constexpr int kRegion = kTileM * 128;         // one 64-column block of a tile
   static constexpr int kOffQ = 0;
-  static constexpr int kOffP = kOffQ + 2 * kTileBytes;
-  static constexpr int kOffKV = kOffP + 2 * kPBytes;
+  static constexpr int kOffKV = kOffQ + 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  // q_full, full[S], empty[S] (K ring slots first, then V ring), s_ready[2], s_free[2],
-  // p_ready[2], pv_done[2], mma_final
-  static constexpr int kNumBars = 1 + 2 * kStages + 9;
+  // q_full, full[S], empty[S], s_ready[2], p_ready[2], o_done[2], mma_final
+  static constexpr int kNumBars = 1 + 2 * kStages + 7;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
 };
@@ -83,10 +82,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* ring_full = bars + 1;
   uint64_t* ring_empty = ring_full + S;
   uint64_t* s_ready = ring_empty + S;
-  uint64_t* s_free = s_ready + 2;
-  uint64_t* p_ready = s_free + 2;
-  uint64_t* pv_done = p_ready + 2;
-  uint64_t* mma_final = pv_done + 2;
+  uint64_t* p_ready = s_ready + 2;
+  uint64_t* o_done = p_ready + 2;
+  uint64_t* mma_final = o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -119,9 +117,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_ready[t], 1);
-      mbar_init(&s_free[t], kTileM);
       mbar_init(&p_ready[t], kTileM);
-      mbar_init(&pv_done[t], 1);
+      mbar_init(&o_done[t], 1);
     }
     mbar_init(mma_final, 1);
     *abort_flag = 0;
@@ -136,6 +133,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx w{abort_flag, p.status, p.wait_budget_ns};
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     regs_dec<kRegsControl, kRegsLaunch>();
@@ -151,63 +149,51 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int z = 0; z < D / 64; ++z)
           tma_load_3d(smem + C::kOffQ + t * C::kTileBytes + z * C::kRegion, &tmQ, q_full, z * 64,
                       q0 + t * kTileM, q_head);
-      // ring r (0 = K, 1 = V): slots [base[r], base[r] + n[r]), cnt[r] tiles pushed so far
-      const int base[2] = {0, C::kStagesK};
-      const int nst[2] = {C::kStagesK, C::kStagesV};
-      int cnt[2] = {0, 0};
-      auto push = [&](int r, int kv_tile) -> bool {
-        const int s = base[r] + cnt[r] % nst[r];
-        const uint32_t ph = (cnt[r] / nst[r]) & 1;
-        if (!mbar_wait(&ring_empty[s], ph ^ 1, w)) return false;
+      int it = 0;
+      auto push = [&](const CUtensorMap* map, int kv_tile) -> bool {
+        const int s = it % S;
+        if (!mbar_wait_spin(&ring_empty[s], ((it / S) & 1) ^ 1, w)) return false;
         mbar_arrive_expect_tx(&ring_full[s], C::kTileBytes);
-        const CUtensorMap* map = r == 0 ? &tmK : &tmV;
 #pragma unroll
         for (int z = 0; z < D / 64; ++z)
           tma_load_3d(smem + C::kOffKV + s * C::kTileBytes + z * C::kRegion, map, &ring_full[s], z * 64,
                       kv_tile * kTileN, kv_head);
-        ++cnt[r];
+        ++it;
         return true;
       };
       bool ok = true;
       for (int j = 0; j < n_kv && ok; ++j) {
-        ok = push(0, j);
-        if (ok && j >= 1) ok = push(1, j - 1);
+        ok = push(&tmK, j);
+        if (ok) ok = push(&tmV, j);
       }
-      if (ok) ok = push(1, n_kv - 1);
       if (!ok) {
         // Error path: let the loads already issued land before the CTA exits.
         WaitCtx drain{abort_flag, p.status, 20000000ull};
         volatile int zero = 0;
         drain.abort_flag = &zero;
-        for (int r = 0; r < 2; ++r)
-          for (int k = max(0, cnt[r] - nst[r]); k < cnt[r]; ++k)
-            mbar_wait(&ring_full[base[r] + k % nst[r]], (k / nst[r]) & 1, drain);
+        for (int k = max(0, it - S); k < it; ++k) mbar_wait(&ring_full[k % S], (k / S) & 1, drain);
         mbar_wait(q_full, 0, drain);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs this role so that descriptors are warp-uniform; lane 0
-    // alone issues tcgen05.mma and tcgen05.commit. Descriptors are built once
-    // and advanced by constant offsets of the start-address field: recomputing
-    // them per MMA from runtime indices halves the issue rate.
+    // alone issues tcgen05.mma and tcgen05.commit. Descriptors are built once and
+    // advanced by constant offsets of the start-address field.
     regs_dec<kRegsControl, kRegsLaunch>();
     const bool leader = lane == 0;
     constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, false, true);
     const uint64_t d_q = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
-    const uint64_t d_p = sdesc_sw128(smem_u32(smem + C::kOffP), 16, 1024);
     const uint64_t d_k = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);           // K-major view
     const uint64_t d_v = sdesc_sw128(smem_u32(smem + C::kOffKV), C::kRegion, 1024);   // MN-major view
-    const int base[2] = {0, C::kStagesK};
-    const int nst[2] = {C::kStagesK, C::kStagesV};
-    int cnt[2] = {0, 0};
-    bool ok = mbar_wait(q_full, 0, w);
+    int cnt = 0;
+    bool ok = mbar_wait_spin(q_full, 0, w);
     tc_fence_after();
-    auto take = [&](int r, int& slot) -> bool {  // next tile of ring r (0 = K, 1 = V)
-      slot = base[r] + cnt[r] % nst[r];
-      const bool res = mbar_wait(&ring_full[slot], (cnt[r] / nst[r]) & 1, w);
-      ++cnt[r];
+    auto take = [&](int& slot) -> bool {  // next stage of the ring
+      slot = cnt % S;
+      const bool res = mbar_wait_spin(&ring_full[slot], (cnt / S) & 1, w);
+      ++cnt;
       tc_fence_after();
       return res;
     };
@@ -217,50 +203,49 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * C::kRegion + (k & 3) * 32;
-        if (leader) mma_bf16_ss(tmem + t * 128, desc_advance(a0, off), desc_advance(b0, off), kIdescS, k > 0 ? 1u : 0u);
+        if (leader)
+          mma_bf16_ss(tmem + t * 128, desc_advance(a0, off), desc_advance(b0, off), kIdescS, k > 0 ? 1u : 0u);
       }
       if (leader) mma_commit(&s_ready[t]);
     };
     auto issue_pv = [&](int t, int slot, int j) {
-      const uint64_t a0 = desc_advance(d_p, t * C::kPBytes);
       const uint64_t b0 = desc_advance(d_v, slot * C::kTileBytes);
 #pragma unroll
-      for (int k = 0; k < kTileN / 16; ++k) {
-        const uint32_t aoff = (k >> 2) * C::kRegion + (k & 3) * 32;
+      for (int k = 0; k < kTileN / 16; ++k)
         if (leader)
-          mma_bf16_ss(tmem + 256 + t * 128, desc_advance(a0, aoff), desc_advance(b0, k * 16 * 128), kIdescPV,
+          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8, desc_advance(b0, k * 16 * 128), kIdescPV,
                       (j > 0 || k > 0) ? 1u : 0u);
-      }
-      if (leader) mma_commit(&pv_done[t]);
     };
-    auto do_pv = [&](int j) -> bool {  // PV_0(j), PV_1(j) from the V_j stage
-      int slot;
-      if (!take(1, slot)) return false;
-      for (int t = 0; t < 2; ++t) {
-        if (j >= n_iter[t]) continue;
-        if (!mbar_wait(&p_ready[t], j & 1, w)) return false;
-        tc_fence_after();
-        issue_pv(t, slot, j);
+    if (ok && n_kv > 0) {
+      int kslot;
+      ok = take(kslot);
+      if (ok) {
+        for (int t = 0; t < 2; ++t)
+          if (n_iter[t] > 0) issue_s(t, kslot);
+        if (leader) mma_commit(&ring_empty[kslot]);
       }
-      if (leader) mma_commit(&ring_empty[slot]);
-      return true;
-    };
+    }
     for (int j = 0; j < n_kv && ok; ++j) {
-      int slot;
-      ok = take(0, slot);
+      int vslot, kslot = -1;
+      if (!(ok = take(vslot))) break;
       for (int t = 0; t < 2 && ok; ++t) {
         if (j >= n_iter[t]) continue;
-        if (j > 0) {
-          ok = mbar_wait(&s_free[t], (j - 1) & 1, w);
-          tc_fence_after();
+        if (!(ok = mbar_wait_spin(&p_ready[t], j & 1, w))) break;
+        tc_fence_after();
+        issue_pv(t, vslot, j);
+        if (j + 1 < n_iter[t]) {
+          if (kslot < 0 && !(ok = take(kslot))) break;
+          issue_s(t, kslot);
+        } else if (leader) {
+          mma_commit(&o_done[t]);
         }
-        if (ok) issue_s(t, slot);
       }
       if (!ok) break;
-      if (leader) mma_commit(&ring_empty[slot]);
-      if (j >= 1) ok = do_pv(j - 1);
+      if (leader) {
+        mma_commit(&ring_empty[vslot]);
+        if (kslot >= 0) mma_commit(&ring_empty[kslot]);
+      }
     }
-    if (ok) ok = do_pv(n_kv - 1);
     // Every MMA issued above must finish before TMEM is released.
     if (leader) mma_commit(mma_final);
     __syncwarp();
@@ -281,14 +266,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
       const uint32_t tS = tmem + lane_off + t * 128;
       const uint32_t tO = tmem + lane_off + 256 + t * 128;
-      const uint32_t p_tile = smem_u32(smem + C::kOffP + t * C::kPBytes);
       const int qrow = q0 + t * kTileM + row;
       const float c = p.scale_log2;
       float m_ref = -INFINITY;  // reference max (raw score units)
       float l = 0.f;
       bool ok = true;
       for (int j = 0; j < n; ++j) {
-        if (!(ok = mbar_wait(&s_ready[t], j & 1, w))) break;
+        if (!(ok = mbar_wait_ns(&s_ready[t], j & 1, w, kConsumerPollNs))) break;
         tc_fence_after();
         float s[kTileN];
 #pragma unroll
@@ -299,8 +283,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
         }
-        tc_fence_before();
-        mbar_arrive(&s_free[t]);
 
         const int k0 = j * kTileN;
         if (p.causal && j == n - 1) {
@@ -351,11 +333,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         f2_unpack(rs2[1], rc, rd);
         l += (ra + rb) + (rc + rd);
 
-        if (j >= 1) {
-          // PV(j-1) must be done: it reads the P buffer and accumulates into O.
-          if (!(ok = mbar_wait(&pv_done[t], (j - 1) & 1, w))) break;
-          tc_fence_after();
-        }
+        // PV(j-1) has completed (the commit of S(j) covers it): O may be rescaled.
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -366,22 +344,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
             tmem_st32(tO + cc * 32, r);
           }
-          tmem_st_wait();
         }
-#pragma unroll
-        for (int z = 0; z < 2; ++z) {
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const int c2 = (z * 64 + ch * 8) / 2;
-            st_shared_v4(p_tile + z * C::kRegion + sw128_offset(row, ch), pk[c2], pk[c2 + 1], pk[c2 + 2],
-                         pk[c2 + 3]);
-          }
+        // P into the first 64 columns of S_t (its scores are in registers now).
+        {
+          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[0]);
+          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[32]);
+          tmem_st32(tS, lo);
+          tmem_st32(tS + 32, hi);
         }
-        fence_async_smem();
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_ready[t]);
       }
-      if (ok && (ok = mbar_wait(&pv_done[t], (n - 1) & 1, w))) {
+      if (ok && (ok = mbar_wait_ns(&o_done[t], 0, w, kConsumerPollNs))) {
         tc_fence_after();
         const float inv_l = 1.f / l;
         const bool valid = qrow < p.N;

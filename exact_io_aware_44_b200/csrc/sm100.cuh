@@ -92,6 +92,80 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   return false;
 }
 
+// Suspension cap of the many-thread consumer waits (softmax / elementwise
+// warpgroups). Without a cap a waiter may sleep far past the phase completion.
+#ifndef FA_CONSUMER_POLL_NS
+#define FA_CONSUMER_POLL_NS 200
+#endif
+constexpr uint32_t kConsumerPollNs = FA_CONSUMER_POLL_NS;
+
+// One poll that may suspend the thread for at most `ns` nanoseconds.
+__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// As mbar_wait, with each suspension capped at `ns` nanoseconds: bounds how
+// long a waiter can sleep past the phase completion while polling rarely.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, const WaitCtx& w, uint32_t ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait_ns(a, parity, ns)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t max_iter = w.budget_ns / 8 + 1024;
+  for (uint64_t i = 0; i < max_iter; ++i) {
+    if (mbar_try_wait_ns(a, parity, ns)) return true;
+    if ((i & 15) == 15) {
+      if (*w.abort_flag) return false;
+      if (globaltimer_ns() - t0 > w.budget_ns) break;
+    }
+  }
+  *w.abort_flag = 1;
+  record_error(w.status, FA_ERR_DEVICE_TIMEOUT);
+  return false;
+}
+
+// Non-suspending probe of a phase (mbarrier.test_wait).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// As mbar_wait, but the thread never suspends: for the single-warp roles (MMA
+// issue, TMA production) whose wake-up latency is on the critical path. A
+// suspended try_wait can sleep on the order of a microsecond past the phase
+// completion, which idles the tensor core; a spinning warp costs only its own
+// issue slots. Many-thread waiters keep mbar_wait.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_test_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t max_iter = w.budget_ns / 8 + 1024;  // every probe takes well over 8 ns
+  for (uint64_t i = 0; i < max_iter; ++i) {
+    if (mbar_test_wait(a, parity)) return true;
+    if ((i & 63) == 63) {
+      if (*w.abort_flag) return false;
+      if (globaltimer_ns() - t0 > w.budget_ns) break;
+    }
+  }
+  *w.abort_flag = 1;
+  record_error(w.status, FA_ERR_DEVICE_TIMEOUT);
+  return false;
+}
+
 // ----------------------------------------------------------------------------
 // proxy / tcgen05 ordering fences
 // ----------------------------------------------------------------------------
@@ -161,6 +235,18 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Same, with the A operand in Tensor Memory (128 lanes = M rows; 32-bit column c
+// holds the bf16 pair k = 2c (low half), 2c + 1; a K = 16 step spans 8 columns).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
