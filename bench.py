@@ -45,7 +45,10 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 # DRAM bytes (read + write) per launch of the dominant kernel from one ncu
 # capture, with the hash of the kernel source it was taken on. A changed
 # source makes the figure stale and the bench reports null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/bwd_main_d128_B2H32N8192_causal.md
+    ("bwd_main", "c3"): {"bytes_per_launch": 809782016 + 490684160, "csrc_sha": "cf77055da08ab318"},
+}
 
 
 def kernel_source_hash(kernel: str) -> str:
