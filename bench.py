@@ -184,17 +184,19 @@ def blas_threads() -> int:
 
 
 def oracle_head_step(w, b: int, h: int):
-    """Forward + backward of one (batch, head) of workload `w` in float64; returns FLOPs."""
+    """Forward (+ backward) of one (batch, head) of workload `w` in float64; returns (seconds, FLOPs)."""
     import numpy as np
     import oracle
     import synth
-    q = synth.head_slice(w, synth.TID_Q, b, h)[None, None]
-    k = synth.head_slice(w, synth.TID_K, b, h // w.group)[None, None]
-    v = synth.head_slice(w, synth.TID_V, b, h // w.group)[None, None]
-    do = synth.head_slice(w, synth.TID_DO, b, h)[None, None]
+    ds = w.descale if w.dtype == "e4m3" else 1.0  # E4M3 slices hold codes; real value = code * descale
+    q = synth.head_slice(w, synth.TID_Q, b, h)[None, None].astype(np.float64) * ds
+    k = synth.head_slice(w, synth.TID_K, b, h // w.group)[None, None].astype(np.float64) * ds
+    v = synth.head_slice(w, synth.TID_V, b, h // w.group)[None, None].astype(np.float64) * ds
+    do = synth.head_slice(w, synth.TID_DO, b, h)[None, None] if w.backward else None
     t0 = time.perf_counter()
     o, lse = oracle.attention_fwd64(q, k, v, w.causal, w.scale)
-    oracle.attention_bwd64(q, k, v, do, w.causal, w.scale, o=o, lse=lse)
+    if w.backward:
+        oracle.attention_bwd64(q, k, v, do, w.causal, w.scale, o=o, lse=lse)
     dt = time.perf_counter() - t0
     f = 4.0 * w.N * w.N * w.d * (0.5 if w.causal else 1.0)
     return dt, f * (3.5 if w.backward else 1.0)
@@ -208,8 +210,9 @@ def cpu_baseline(w, budget_s: float = 15.0):
         total_t += dt
         total_f += f
         heads += 1
+    what = "forward + backward" if w.backward else "forward"
     return {"value": total_f / total_t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{heads} of {w.B * w.Hq} (batch, head) pairs, full forward + backward each, float64 NumPy",
+            "sample": f"{heads} of {w.B * w.Hq} (batch, head) pairs, full {what} each, float64 NumPy",
             "seconds": round(total_t, 3)}
 
 
@@ -227,7 +230,10 @@ def run_ours(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
-    peak = float(peaks["bf16_tflops"])
+    fp8 = w.dtype == "e4m3"
+    # dense FP8 peak = measured bf16 x the nominal 2x (4.5 vs 2.25 PFLOP/s dense)
+    peak_mul = 2.0 if fp8 else 1.0
+    peak = float(peaks["bf16_tflops"]) * peak_mul
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
 
@@ -237,25 +243,33 @@ def run_ours(args, w, world, rank, local):
 
     # inputs: generated on the host (seeded), kept pinned for the e2e leg
     host = {}
-    for name, tid in (("q", synth.TID_Q), ("k", synth.TID_K), ("v", synth.TID_V), ("do", synth.TID_DO)):
-        host[name] = torch.from_numpy(synth.tensor(w, tid)).to(torch.bfloat16).pin_memory()
+    tids = (("q", synth.TID_Q), ("k", synth.TID_K), ("v", synth.TID_V)) + ((("do", synth.TID_DO),) if w.backward else ())
+    in_dtype = torch.float8_e4m3fn if fp8 else torch.bfloat16
+    for name, tid in tids:
+        host[name] = torch.from_numpy(synth.tensor(w, tid)).to(in_dtype).pin_memory()
     d_in = {n: t.to(dev) for n, t in host.items()}
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
     o = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
-    dq = torch.empty_like(o)
-    dk = torch.empty((B, Hkv, N, d), dtype=torch.bfloat16, device=dev)
-    dv = torch.empty_like(dk)
-    ws = torch.empty(fa.workspace_bytes(B, Hq, Hkv, N, d), dtype=torch.uint8, device=dev)
+    if w.backward:
+        dq = torch.empty_like(o)
+        dk = torch.empty((B, Hkv, N, d), dtype=torch.bfloat16, device=dev)
+        dv = torch.empty_like(dk)
+        ws = torch.empty(fa.workspace_bytes(B, Hq, Hkv, N, d), dtype=torch.uint8, device=dev)
     P = lambda t: t.data_ptr()
 
     def step(events=None):
         if events is not None:
             events[0].record(stream)
-        rc = fa.fwd_raw(P(d_in["q"]), P(d_in["k"]), P(d_in["v"]), P(o), P(lse), B, Hq, Hkv, N, d, w.causal,
-                        w.scale, sp)
+        if fp8:
+            ds = w.descale
+            rc = fa.fwd_fp8_raw(P(d_in["q"]), P(d_in["k"]), P(d_in["v"]), ds, ds, ds, P(o), P(lse), B, Hq, Hkv, N, d,
+                                w.causal, w.scale, sp)
+        else:
+            rc = fa.fwd_raw(P(d_in["q"]), P(d_in["k"]), P(d_in["v"]), P(o), P(lse), B, Hq, Hkv, N, d, w.causal,
+                            w.scale, sp)
         if rc:
-            raise fa.FAError(rc, "fa_fwd")
+            raise fa.FAError(rc, "fa_fwd_fp8" if fp8 else "fa_fwd")
         if not w.backward:
             if events is not None:
                 for e in events[1:]:
@@ -317,16 +331,19 @@ def run_ours(args, w, world, rank, local):
         traffic = rec["bytes_per_launch"]
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": UNIT,
                 "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": dominant,
-                "peak_source": f"{peak_src} dense bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
-                if peak_src == "measured" else "fallback 1.59 PFLOP/s",
-                "frac_of_sustained": round(achieved / float(peaks.get("bf16_tflops_sustained", peak)), 4)}
+                "peak_source": (f"{peak_src} dense bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
+                                if peak_src == "measured" else "fallback 1.59 PFLOP/s")
+                + (" x 2, the nominal dense fp8:bf16 ratio" if fp8 else ""),
+                "frac_of_sustained": round(achieved / (float(peaks.get("bf16_tflops_sustained", peak)) * peak_mul),
+                                           4)}
 
     # ---------------------------------------------------- end to end (host buffers)
     e2e = None
     if not args.no_e2e:
-        out_host = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                    for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
-        dev_out = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+        dev_out = {"o": o, "lse": lse}
+        if w.backward:
+            dev_out.update(dq=dq, dk=dk, dv=dv)
+        out_host = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in dev_out.items()}
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = sum(t.numel() * t.element_size() for t in out_host.values())
         Ke = max(1, min(K, args.e2e_steps))
@@ -356,13 +373,14 @@ def run_ours(args, w, world, rank, local):
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": f"{w.name}: B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} "
-                               f"{'causal' if w.causal else 'non-causal'} bf16 "
+                               f"{'causal' if w.causal else 'non-causal'} {w.dtype} "
                                f"{'fwd+bwd' if w.backward else 'fwd'}",
                    "B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "causal": w.causal,
-                   "l2": "inputs larger than L2 (Q, K, V, O, dO are "
-                         f"{B * Hq * N * d * 2 / 1e6:.0f} MB each; L2 is 126 MB)",
+                   "l2": "inputs larger than L2 ("
+                         + ("Q, K, V, O, dO are" if w.backward else "Q, K, V are")
+                         + f" {B * Hq * N * d * (1 if fp8 else 2) / 1e6:.0f} MB each; L2 is 126 MB)",
                    "parallelism": f"replicas x{world}"},
         "pct_of_peak": round(100 * value / world / peak, 2),
         "fwd_tflops": round(kernels["fwd"]["tflops"], 1),
@@ -392,12 +410,14 @@ def run_reference(args, w):
             flops = f
     ms = 1e3 * statistics.mean(times)
     value = flops / (ms / 1e3) / 1e12
-    sample = f"one (batch, head) pair per step: full forward + backward of B=1 H=1 N={w.N} d={w.d} in float64"
+    what = "forward + backward" if w.backward else "forward"
+    sample = f"one (batch, head) pair per step: full {what} of B=1 H=1 N={w.N} d={w.d} in float64"
     return {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": 0, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} "
-                                   f"{'causal' if w.causal else 'non-causal'} fwd+bwd (sampled per step)"},
+                                   f"{'causal' if w.causal else 'non-causal'} {w.dtype} "
+                                   f"{'fwd+bwd' if w.backward else 'fwd'} (sampled per step)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": blas_threads(),
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -409,7 +429,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c3", help="c2, c3, c4 (forward only) or c5")
+    ap.add_argument("--workload", default="c3",
+                    help="c2, c3, c5 (bf16 fwd+bwd), c4 (bf16 fwd), f3, f4 (E4M3 fwd)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")

@@ -89,18 +89,20 @@ int check_sizes(int B, int Hq, int Hkv, int N, int d, float scale, bool* empty) 
   return FA_OK;
 }
 
-// 3-D bf16 tensor map over [heads, N, d] with a 64-column x `box_rows` box and
-// the 128-byte swizzle; rows past N read as zero.
-int make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box_rows = kTileM) {
+// 3-D tensor map over [heads, N, d] (bf16, or E4M3 as bytes) with a box one
+// 128-byte block wide and `box_rows` high, and the 128-byte swizzle; rows past N
+// read as zero.
+int make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box_rows = kTileM, bool e4m3 = false) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return FA_ERR_LAUNCH;
+  const cuuint64_t elem = e4m3 ? 1 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)heads};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)d * elem, (cuuint64_t)N * d * elem};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / elem), (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -158,8 +160,45 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.causal = causal ? 1 : 0;
   p.n_qblk = (N + 2 * kTileM - 1) / (2 * kTileM);
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_scale = 1.f;
   p.wait_budget_ns = g_wait_budget_ns.load();
   if (launch_fwd_bf16(tq, tk, tv, p, d, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, float descale_k, float descale_v,
+               void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  bool empty;
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
+  if (rc != FA_OK) return rc;
+  for (float ds : {descale_q, descale_k, descale_v})
+    if (!(ds > 0.f) || !isfinite(ds)) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  const float c = scale * descale_q * descale_k * 1.4426950408889634f;
+  if (!isfinite(c) || !(c > 0.f) || !isfinite(descale_v)) return FA_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  if ((rc = current_device(&di)) != FA_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_map(&tq, q, d, N, B * Hq, kTileM, true)) != FA_OK) return rc;
+  if ((rc = make_map(&tk, k, d, N, B * Hkv, kTileM, true)) != FA_OK) return rc;
+  if ((rc = make_map(&tv, v, d, N, B * Hkv, kTileM, true)) != FA_OK) return rc;
+  FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.status = di->status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.causal = causal ? 1 : 0;
+  p.n_qblk = (N + 2 * kTileM - 1) / (2 * kTileM);
+  p.scale_log2 = c;
+  p.o_scale = descale_v;
+  p.wait_budget_ns = g_wait_budget_ns.load();
+  if (launch_fwd_e4m3(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
 }
 

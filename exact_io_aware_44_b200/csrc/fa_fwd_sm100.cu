@@ -1,4 +1,4 @@
-// fa_fwd_sm100.cu -- bf16 attention forward on sm_100a tensor cores.
+// fa_fwd_sm100.cu -- attention forward on sm_100a tensor cores (bf16, or E4M3 inputs).
 //
 // The method is the tiled forward with the online softmax: each query tile
 // streams the key/value tiles through on-chip memory, keeps a running row max m
@@ -17,6 +17,12 @@
 //   warps 8-11  softmax for query tile 1.
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 [384,384+d);
 // P_t (bf16 pairs, 64 columns) overwrites the first half of S_t once it is read.
+//
+// E4M3 inputs (d = 128) run the same kernel with kind::f8f6f4 MMAs: a tile is
+// 16 KB (one 128-byte swizzle block wide), the ring holds 10 stages, an MMA
+// steps 32 elements of K, and P is rounded to E4M3, four keys per TMEM column
+// (32 columns). The Q and K descales fold into c; V's descale multiplies the
+// final 1/l.
 //
 // Per key tile j, a softmax thread loads its row of S_t, applies the causal
 // mask on the diagonal tile, updates the running max, and computes
@@ -51,11 +57,18 @@ constexpr int kRegsSoftmax = 208;
 static_assert(kFwdThreads * kRegsLaunch == 128 * kRegsControl + 256 * kRegsSoftmax, "register split");
 constexpr uint32_t kRescaleThresholdLog2 = 8;  // rescale only when m grows by > 2^8
 
-template <int D>
+// D: head dim; FP8: E4M3 Q, K, V and P (kind::f8f6f4 MMAs), else bf16 (kind::f16).
+template <int D, bool FP8>
 struct FwdCfg {
-  static constexpr int kStages = (D == 128) ? 5 : 10;  // K/V ring, in order K_0, V_0, K_1, V_1, ...
-  static constexpr int kTileBytes = kTileM * D * 2;    // one Q, K or V tile (bf16)
-  static constexpr int kRegion = kTileM * 128;         // one 64-column block of a tile
+  static constexpr int kElem = FP8 ? 1 : 2;                      // bytes per element
+  static constexpr int kStages = (FP8 || D == 64) ? 10 : 5;      // K/V ring: K_0, V_0, K_1, V_1, ...
+  static constexpr int kTileBytes = kTileM * D * kElem;          // one Q, K or V tile
+  static constexpr int kRegion = kTileM * 128;                   // one 128-byte-wide column block
+  static constexpr int kRegions = D * kElem / 128;               // column blocks per tile
+  static constexpr int kBoxCols = 128 / kElem;                   // elements per block row
+  static constexpr int kKStep = 32 / kElem;                      // K per MMA (32 bytes of each row)
+  static constexpr int kSSteps = D / kKStep;                     // MMAs per S tile
+  static constexpr int kPvSteps = kTileN / kKStep;               // MMAs per P V (8 TMEM columns each)
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kOffQ + 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
@@ -69,11 +82,11 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int D>
+template <int D, bool FP8>
 __global__ void __launch_bounds__(kFwdThreads, 1)
-    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, FP8>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -146,8 +159,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_arrive_expect_tx(q_full, n_qt * C::kTileBytes);
       for (int t = 0; t < n_qt; ++t)
 #pragma unroll
-        for (int z = 0; z < D / 64; ++z)
-          tma_load_3d(smem + C::kOffQ + t * C::kTileBytes + z * C::kRegion, &tmQ, q_full, z * 64,
+        for (int z = 0; z < C::kRegions; ++z)
+          tma_load_3d(smem + C::kOffQ + t * C::kTileBytes + z * C::kRegion, &tmQ, q_full, z * C::kBoxCols,
                       q0 + t * kTileM, q_head);
       int it = 0;
       auto push = [&](const CUtensorMap* map, int kv_tile) -> bool {
@@ -155,8 +168,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!mbar_wait_spin(&ring_empty[s], ((it / S) & 1) ^ 1, w)) return false;
         mbar_arrive_expect_tx(&ring_full[s], C::kTileBytes);
 #pragma unroll
-        for (int z = 0; z < D / 64; ++z)
-          tma_load_3d(smem + C::kOffKV + s * C::kTileBytes + z * C::kRegion, map, &ring_full[s], z * 64,
+        for (int z = 0; z < C::kRegions; ++z)
+          tma_load_3d(smem + C::kOffKV + s * C::kTileBytes + z * C::kRegion, map, &ring_full[s], z * C::kBoxCols,
                       kv_tile * kTileN, kv_head);
         ++it;
         return true;
@@ -182,8 +195,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // advanced by constant offsets of the start-address field.
     regs_dec<kRegsControl, kRegsLaunch>();
     const bool leader = lane == 0;
-    constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
-    constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, false, true);
+    constexpr uint32_t kIdescS =
+        FP8 ? idesc_e4m3_f32(kTileM, kTileN, false, false) : idesc_bf16_f32(kTileM, kTileN, false, false);
+    constexpr uint32_t kIdescPV = FP8 ? idesc_e4m3_f32(kTileM, D, false, true) : idesc_bf16_f32(kTileM, D, false, true);
     const uint64_t d_q = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
     const uint64_t d_k = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);           // K-major view
     const uint64_t d_v = sdesc_sw128(smem_u32(smem + C::kOffKV), C::kRegion, 1024);   // MN-major view
@@ -201,20 +215,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint64_t a0 = desc_advance(d_q, t * C::kTileBytes);
       const uint64_t b0 = desc_advance(d_k, slot * C::kTileBytes);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
+      for (int k = 0; k < C::kSSteps; ++k) {
         const uint32_t off = (k >> 2) * C::kRegion + (k & 3) * 32;
-        if (leader)
-          mma_bf16_ss(tmem + t * 128, desc_advance(a0, off), desc_advance(b0, off), kIdescS, k > 0 ? 1u : 0u);
+        if (leader) {
+          if constexpr (FP8)
+            mma_e4m3_ss(tmem + t * 128, desc_advance(a0, off), desc_advance(b0, off), kIdescS, k > 0 ? 1u : 0u);
+          else
+            mma_bf16_ss(tmem + t * 128, desc_advance(a0, off), desc_advance(b0, off), kIdescS, k > 0 ? 1u : 0u);
+        }
       }
       if (leader) mma_commit(&s_ready[t]);
     };
     auto issue_pv = [&](int t, int slot, int j) {
       const uint64_t b0 = desc_advance(d_v, slot * C::kTileBytes);
 #pragma unroll
-      for (int k = 0; k < kTileN / 16; ++k)
-        if (leader)
-          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8, desc_advance(b0, k * 16 * 128), kIdescPV,
-                      (j > 0 || k > 0) ? 1u : 0u);
+      for (int k = 0; k < C::kPvSteps; ++k) {
+        if (leader) {
+          const uint64_t bk = desc_advance(b0, k * C::kKStep * 128);
+          if constexpr (FP8)
+            mma_e4m3_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8, bk, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+          else
+            mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8, bk, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+        }
+      }
     };
     if (ok && n_kv > 0) {
       int kslot;
@@ -318,15 +341,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           rescale = true;
         }
         const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-        // P = 2^(S c - m c), packed to bf16 pairs at once; l sums the fp32 values.
-        uint32_t pk[kTileN / 2];
+        // P = 2^(S c - m c), packed at once (bf16 pairs, or E4M3 quads: one TMEM column
+        // each); l sums the fp32 values. P <= 2^8 fits E4M3; E4M3 flushes P < 2^-10 to zero.
+        uint32_t pk[kTileN / (FP8 ? 4 : 2)];
         uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-        for (int i = 0; i < kTileN; i += 2) {
+        for (int i = 0; i < kTileN; i += 4) {
           const float e0 = ex2(fmaf(s[i], c, -mc));
           const float e1 = ex2(fmaf(s[i + 1], c, -mc));
-          rs2[(i >> 1) & 1] = f2_add(rs2[(i >> 1) & 1], f2_pack(e0, e1));
-          pk[i / 2] = pack_bf16x2(e0, e1);
+          const float e2 = ex2(fmaf(s[i + 2], c, -mc));
+          const float e3 = ex2(fmaf(s[i + 3], c, -mc));
+          rs2[0] = f2_add(rs2[0], f2_pack(e0, e1));
+          rs2[1] = f2_add(rs2[1], f2_pack(e2, e3));
+          if constexpr (FP8) {
+            pk[i / 4] = pack_e4m3x4(e0, e1, e2, e3);
+          } else {
+            pk[i / 2] = pack_bf16x2(e0, e1);
+            pk[i / 2 + 1] = pack_bf16x2(e2, e3);
+          }
         }
         float ra, rb, rc, rd;
         f2_unpack(rs2[0], ra, rb);
@@ -345,8 +377,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_st32(tO + cc * 32, r);
           }
         }
-        // P into the first 64 columns of S_t (its scores are in registers now).
-        {
+        // P into the first columns of S_t (its scores are in registers now).
+        if constexpr (FP8) {
+          tmem_st32(tS, pk);
+        } else {
           uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[0]);
           uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[32]);
           tmem_st32(tS, lo);
@@ -358,7 +392,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (ok && (ok = mbar_wait_ns(&o_done[t], 0, w, kConsumerPollNs))) {
         tc_fence_after();
-        const float inv_l = 1.f / l;
+        const float inv_l = p.o_scale / l;
         const bool valid = qrow < p.N;
         const size_t row_idx = (size_t)(b * p.Hq + h) * p.N + qrow;
         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row_idx * D);
@@ -393,20 +427,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool FP8>
 cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                          cudaStream_t stream) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, FP8>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   const long long grid = (long long)p.B * p.Hq * p.n_qblk;
-  fwd_bf16_kernel<D><<<(unsigned)grid, kFwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  fwd_kernel<D, FP8><<<(unsigned)grid, kFwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -414,7 +448,12 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int d, cudaStream_t s) {
-  return d == 128 ? launch_fwd_d<128>(tq, tk, tv, p, s) : launch_fwd_d<64>(tq, tk, tv, p, s);
+  return d == 128 ? launch_fwd_d<128, false>(tq, tk, tv, p, s) : launch_fwd_d<64, false>(tq, tk, tv, p, s);
+}
+
+cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, cudaStream_t s) {
+  return launch_fwd_d<128, true>(tq, tk, tv, p, s);
 }
 
 }  // namespace fa

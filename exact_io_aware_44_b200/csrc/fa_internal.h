@@ -18,7 +18,8 @@ struct FwdParams {
   int B, Hq, Hkv, N;
   int causal;
   int n_qblk;         // query blocks of 2 tiles (256 rows) per head
-  float scale_log2;   // scale * log2(e)
+  float scale_log2;   // scale * log2(e) (times the Q and K descales for E4M3 inputs)
+  float o_scale;      // multiplies O at the end (the V descale for E4M3 inputs, else 1)
   uint64_t wait_budget_ns;
 };
 
@@ -48,6 +49,8 @@ struct BwdParams {
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int d, cudaStream_t s);
+cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, cudaStream_t s);
 cudaError_t launch_fwd_f32(const FwdF32Params& p, cudaStream_t s);
 // Backward phases: D and zeroed dQ accumulator; main kernel; dQ conversion.
 cudaError_t launch_bwd_preprocess(const BwdParams& p, cudaStream_t s);

@@ -76,6 +76,29 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * fa_fwd_fp8 -- forward pass with E4M3 inputs (8-bit tensor cores).
+ *
+ * The third FlashAttention generation adds an FP8 path (E4M3 and E5M2) worth
+ * a further 1.5-2x (FlashAttention family short answer, second paragraph, and
+ * the version table on the same page). This call computes the forward of
+ * fa_fwd on inputs stored as E4M3 bytes with one scale per tensor, whose real
+ * values are
+ *   Q = descale_q * q,  K = descale_k * k,  V = descale_v * v,
+ * and O = softmax(scale * Q K^T) V, lse = m + ln(l) as in fa_fwd.
+ *   q [B,Hq,N,d], k/v [B,Hkv,N,d]  E4M3 bytes (OCP FP8, finite max 448), read only
+ *   descale_q/k/v                  positive finite float scales
+ *   o [B,Hq,N,d] bf16, lse [B,Hq,N] float32  outputs, as in fa_fwd
+ *   d must be 128. Arithmetic: E4M3 products with fp32 accumulation for S and
+ *   for P V; the probabilities P are rounded to E4M3 (values below 2^-10 of the
+ *   tile's reference maximum become 0) before the P V product, while the row
+ *   sums l add the unrounded fp32 values.
+ * Returns the codes of fa_fwd; FA_ERR_INVALID_ARG also for a descale that is
+ * not positive and finite.
+ */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, float descale_k, float descale_v,
+               void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
+
+/*
  * fa_fwd_f32 -- float32 forward pass (CUDA cores, fp32 throughout).
  *
  * The same computation as fa_fwd, on float32 q, k, v and o. Tiles of queries

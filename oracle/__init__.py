@@ -12,6 +12,8 @@ Parity status per function (what pins it; see tests/test_oracle.py):
   online_softmax_trace64  pinned: equals the one-pass softmax on adversarial rows.
   head_fwd64 / group_bwd_sampled64
                           pinned: equal the full oracle restricted to the sampled rows.
+  head_probs64            pinned: SciPy softmax of brute-force scores, zero above the
+                          causal diagonal, P V reproduces the brute-force output.
   finite_diff_grads64     pinned: exact gradients of closed-form cases.
 The pages print no worked numeric example, so no value is pinned to a printed number.
 """
@@ -23,5 +25,6 @@ from .attention64 import (  # noqa: F401
     finite_diff_grads64,
     group_bwd_sampled64,
     head_fwd64,
+    head_probs64,
     online_softmax_trace64,
 )

@@ -87,6 +87,19 @@ def head_fwd64(qh, kh, vh, causal, scale, rows=None):
     return o, lse
 
 
+def head_probs64(qh, kh, causal, scale, rows=None):
+    """The attention probabilities P = softmax(scale q k^T) of one head, for the
+    given query rows ([R, N]; masked keys are 0). Used to model the rounding of
+    low-precision kernels, whose error depends on the individual P_ij."""
+    qh, kh = _f64(qh), _f64(kh)
+    if rows is None:
+        rows = np.arange(qh.shape[0])
+    rows = np.asarray(rows, dtype=np.int64)
+    s = np.vstack([_scores(qh[i:i + 1], kh, scale, int(i), causal) for i in rows]) if rows.size else \
+        np.zeros((0, kh.shape[0]))
+    return _softmax_rows(s)[0]
+
+
 def attention_fwd64(q, k, v, causal, scale=None):
     """Exact attention. q [B, Hq, N, d]; k, v [B, Hkv, N, d] -> O [B, Hq, N, d], LSE [B, Hq, N]."""
     q, k, v = _f64(q), _f64(k), _f64(v)

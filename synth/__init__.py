@@ -10,7 +10,11 @@ regenerated on its own, which lets the oracle rebuild only the heads it
 samples. Values are iid N(0, 1) float32, multiplied by `std`. For bf16
 workloads they are then rounded to the nearest bf16, ties to even, so the
 GPU and the oracle receive bit-identical numbers. The oracle upcasts them
-exactly to float64.
+exactly to float64. For E4M3 workloads the values are divided by a static
+per-tensor descale (8 std / 448, so that 8 standard deviations map to the
+largest finite E4M3 value) and rounded to the nearest E4M3 value, ties to even,
+saturating at +-448; the slice then holds those codes, and the real input is
+code * descale (exact in float64).
 
 Workloads (shapes from the pages' long-context regime; all synthetic, no dataset):
   c1  fp32 fwd,  B=1 H=1 N=128 d=64, non-causal
@@ -18,6 +22,8 @@ Workloads (shapes from the pages' long-context regime; all synthetic, no dataset
   c3  bf16 fwd+bwd, B=2 H=32 N=8192 d=128, causal, std 1/sqrt(2)
   c4  bf16 fwd,  B=1 H=16 N=65536 d=128, causal
   c5  bf16 fwd+bwd GQA, B=1 Hq=32 Hkv=8 N=32768 d=128, causal
+  f3  E4M3 fwd,  B=2 H=32 N=8192 d=128, causal, std 1/sqrt(2) (c3's shape)
+  f4  E4M3 fwd,  B=1 H=16 N=65536 d=128, causal (c4's shape)
 """
 from __future__ import annotations
 
@@ -41,7 +47,7 @@ class Workload:
     N: int
     d: int
     causal: bool
-    dtype: str  # "f32" or "bf16"
+    dtype: str  # "f32", "bf16" or "e4m3"
     backward: bool
     seed: int
     std: float = 1.0
@@ -58,6 +64,11 @@ class Workload:
     @property
     def group(self) -> int:
         return self.Hq // self.Hkv
+
+    @property
+    def descale(self) -> float:
+        """E4M3 workloads: the float32 value that multiplies every stored code."""
+        return float(np.float32(8.0 * self.std / 448.0))
 
     def fwd_flops(self) -> float:
         f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
@@ -79,7 +90,29 @@ WORKLOADS = {
     "c5": Workload("c5", 1, 32, 8, 32768, 128, True, "bf16", True, 1005,
                    sample_heads=((0, 0), (0, 1), (0, 2), (0, 3),
                                  (0, 28), (0, 29), (0, 30), (0, 31)), sample_rows=256),
+    "f3": Workload("f3", 2, 32, 32, 8192, 128, True, "e4m3", False, 1006,
+                   std=1.0 / math.sqrt(2.0),
+                   sample_heads=((0, 0), (0, 17), (1, 6), (1, 31)), sample_rows=256),
+    "f4": Workload("f4", 1, 16, 16, 65536, 128, True, "e4m3", False, 1007,
+                   sample_heads=((0, 0), (0, 5), (0, 10), (0, 15)), sample_rows=256),
 }
+
+E4M3_MAX = 448.0
+
+
+def round_to_e4m3(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest E4M3 value (OCP FP8: 3 mantissa bits,
+    exponent bias 7, subnormal step 2^-9, no infinities), ties to even,
+    saturating at +-448. Returns float32."""
+    x = np.ascontiguousarray(x, dtype=np.float32).astype(np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)           # below 2^-6 the step stays 2^-9 (subnormals)
+    step = np.exp2(e - 3.0)
+    r = np.round(a / step) * step     # numpy rounds halves to even
+    r = np.minimum(r, E4M3_MAX)
+    return (np.sign(x) * r).astype(np.float32)
 
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
@@ -113,6 +146,8 @@ def head_slice(w: Workload, tid: int, b: int, h: int, n: int | None = None) -> n
         x[rows] *= np.float32(w.spike_mul)
     if w.dtype == "bf16":
         x = round_to_bf16(x)
+    elif w.dtype == "e4m3":
+        x = round_to_e4m3(x / np.float32(w.descale))
     return x
 
 

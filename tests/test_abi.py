@@ -65,6 +65,22 @@ def test_invalid_arguments_rejected_on_host():
     assert _fwd(B=1 << 12, Hq=1 << 10, Hkv=1, N=1 << 10) == -2   # B*Hq*N >= 2^31
 
 
+def _fwd8(d=128, N=128, ds=(0.01, 0.02, 0.03), ptr=0x1000, scale=0.088):
+    return fa.fwd_fp8_raw(ptr, ptr, ptr, *ds, ptr, ptr, 1, 2, 1, N, d, 1, scale, 0)
+
+
+def test_fp8_forward_rejects_bad_arguments_on_host():
+    assert _fwd8(d=64) == -2                      # E4M3 path: d = 128 only
+    assert _fwd8(ds=(0.0, 0.02, 0.03)) == -1      # descales must be positive and finite
+    assert _fwd8(ds=(0.01, -1.0, 0.03)) == -1
+    assert _fwd8(ds=(0.01, 0.02, float("inf"))) == -1
+    assert _fwd8(ds=(0.01, float("nan"), 0.03)) == -1
+    assert _fwd8(ds=(1e30, 1e30, 1.0)) == -1      # scale * descale_q * descale_k overflows
+    assert _fwd8(scale=0.0) == -1
+    assert _fwd8(ptr=0x1004) == -3
+    assert _fwd8(N=0, ptr=0) == 0
+
+
 def test_bwd_rejects_bad_arguments_on_host():
     p = 0x1000
     r = fa.bwd_raw(p, p, p, p, p, p, p, p, p, p + 16, 1, 2, 1, 128, 64, 1, 0.125, 0)

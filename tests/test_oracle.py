@@ -281,6 +281,42 @@ def test_synth_bf16_rounding_matches_torch():
     assert np.array_equal(ours, ref)
 
 
+def test_head_probs_are_the_softmax_of_brute_force_scores():
+    N, d, scale = 37, 8, 0.4
+    q, k, v = rand((N, d), 41), rand((N, d), 42), rand((N, d), 43)
+    for causal in (False, True):
+        rows = np.array([0, 1, 5, 36]) if causal else None
+        p = oracle.head_probs64(q, k, causal, scale, rows=rows)
+        sel = np.arange(N) if rows is None else rows
+        s = scale * np.einsum("id,jd->ij", q[sel], k)
+        if causal:
+            s = np.where(np.arange(N)[None, :] <= sel[:, None], s, -np.inf)
+            assert np.all(p[np.arange(N)[None, :] > sel[:, None]] == 0.0)
+        np.testing.assert_allclose(p, scipy.special.softmax(s, axis=1), rtol=1e-12, atol=1e-15)
+        o_ref, _ = A.attention_naive_loops([q[i].tolist() for i in range(N)], k.tolist(), v.tolist(), causal, scale)
+        np.testing.assert_allclose(p @ v, np.array(o_ref)[sel], rtol=1e-10, atol=1e-12)
+
+
+def test_synth_e4m3_rounding_matches_torch():
+    import torch
+    x = np.random.default_rng(6).standard_normal(20000).astype(np.float32)
+    x *= np.repeat(np.float32([1e-3, 0.05, 1.0, 40.0]), 5000)
+    x[:6] = [2.0 ** -10, 3 * 2.0 ** -11, 1.0625, 1.1875, 448.0, -440.0]  # ties (to even) and the top
+    ours = synth.round_to_e4m3(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float32).numpy()
+    assert np.array_equal(ours, ref)
+    assert synth.round_to_e4m3(np.float32([1000.0, -1e6]))[0] == 448.0   # saturates
+    assert synth.round_to_e4m3(np.float32([-1e6]))[0] == -448.0
+
+
+def test_synth_e4m3_workload_codes():
+    w = synth.WORKLOADS["f3"]
+    x = synth.head_slice(w, synth.TID_K, 1, 5, n=2048)
+    assert np.array_equal(x, synth.round_to_e4m3(x))          # stored values are E4M3 codes
+    deq = x.astype(np.float64) * w.descale
+    assert abs(deq.std() - w.std) < 0.02 and np.abs(x).max() <= 448.0
+
+
 def test_synth_spiked_rows():
     w = synth.WORKLOADS["c2"]
     q = synth.head_slice(w, synth.TID_Q, 1, 3)
