@@ -56,6 +56,12 @@ constexpr int kRegsControl = 88;
 constexpr int kRegsSoftmax = 208;
 static_assert(kFwdThreads * kRegsLaunch == 128 * kRegsControl + 256 * kRegsSoftmax, "register split");
 constexpr uint32_t kRescaleThresholdLog2 = 8;  // rescale only when m grows by > 2^8
+#ifndef FA_FWD_POLY_PAIRS
+#define FA_FWD_POLY_PAIRS 0
+#endif
+// Of every 8 key pairs, how many take 2^x by polynomial on the FMA pipe instead
+// of the SFU (0 = all on the SFU).
+constexpr int kPolyPairs = FA_FWD_POLY_PAIRS;
 
 // D: head dim; FP8: E4M3 Q, K, V and P (kind::f8f6f4 MMAs), else bf16 (kind::f16).
 template <int D, bool FP8>
@@ -345,12 +351,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // each); l sums the fp32 values. P <= 2^8 fits E4M3; E4M3 flushes P < 2^-10 to zero.
         uint32_t pk[kTileN / (FP8 ? 4 : 2)];
         uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        const uint64_t c2 = f2_pack(c, c), nmc2 = f2_pack(-mc, -mc);
 #pragma unroll
         for (int i = 0; i < kTileN; i += 4) {
-          const float e0 = ex2(fmaf(s[i], c, -mc));
-          const float e1 = ex2(fmaf(s[i + 1], c, -mc));
-          const float e2 = ex2(fmaf(s[i + 2], c, -mc));
-          const float e3 = ex2(fmaf(s[i + 3], c, -mc));
+          // x = S c - m c for four keys (two packed FMAs), then 2^x: on the SFU, or for
+          // kPolyPairs of every 8 key pairs by the polynomial on the FMA pipe.
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(s[i], s[i + 1]), c2, nmc2), x0, x1);
+          f2_unpack(f2_fma(f2_pack(s[i + 2], s[i + 3]), c2, nmc2), x2, x3);
+          float e0, e1, e2, e3;
+          if (((i / 2) & 7) < kPolyPairs) {
+            ex2_poly2(x0, x1, e0, e1);
+          } else {
+            e0 = ex2(x0);
+            e1 = ex2(x1);
+          }
+          if (((i / 2 + 1) & 7) < kPolyPairs) {
+            ex2_poly2(x2, x3, e2, e3);
+          } else {
+            e2 = ex2(x2);
+            e3 = ex2(x3);
+          }
           rs2[0] = f2_add(rs2[0], f2_pack(e0, e1));
           rs2[1] = f2_add(rs2[1], f2_pack(e2, e3));
           if constexpr (FP8) {
