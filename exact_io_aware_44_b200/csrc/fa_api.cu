@@ -270,7 +270,7 @@ int run_bwd(int phases, const void* q, const void* k, const void* v, const void*
   if ((rc = current_device(&di)) != FA_OK) return rc;
   CUtensorMap tq, tk, tv, tdo;
   if (main) {
-    const int q_rows = (d == 128) ? 64 : 128;  // query rows per backward tile
+    const int q_rows = bwd_query_rows(d);  // query rows per backward tile
     if ((rc = make_map(&tq, q, d, N, B * Hq, q_rows)) != FA_OK) return rc;
     if ((rc = make_map(&tk, k, d, N, B * Hkv)) != FA_OK) return rc;
     if ((rc = make_map(&tv, v, d, N, B * Hkv)) != FA_OK) return rc;

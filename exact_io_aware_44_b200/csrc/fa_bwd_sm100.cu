@@ -50,6 +50,11 @@ namespace fa {
 namespace {
 
 constexpr int kBwdThreads = 512;
+#ifndef FA_BWD128_ROWS128
+#define FA_BWD128_ROWS128 1
+#endif
+// d = 128: 128-row query tiles (bwd_main_d128_kernel) instead of 64-row ones.
+constexpr bool kBwd128Rows = FA_BWD128_ROWS128 != 0;
 // Register split: the launch gives 128 per thread (512 x 128 = 65536). The
 // control and dQ warpgroups lower to 96 and the two P/dS warpgroups raise to
 // 160: 128 x (96 + 2 x 160 + 96) = 65536.
@@ -169,7 +174,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   using C = BwdCfg<D>;
   constexpr int BR = C::BR;
   constexpr int ST = C::kStages;
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align1024b(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* kv_full = bars;
@@ -571,6 +576,463 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// main backward kernel, d = 128, 128-row query tiles
+// ---------------------------------------------------------------------------
+// With 128 query rows per tile every MMA has M = N = 128 (an N = 64 MMA runs at
+// about half the rate). Tensor Memory then holds exactly S^T [0,128),
+// dP^T [128,256), dV [256,384) and dK [384,512); the dQ tile of query tile i
+// (dQ^T = K^T dS^T, head-dim columns in TMEM lanes) reuses the dP^T columns once dP^T(i) has
+// been read, and dP^T(i+1) is issued once dQ(i) has been read. Shared memory
+// (226 KB): K, V, two Q slots (with -LSE log2 e and D per row), one dO slot, and
+// the P^T and dS^T tiles. The budget leaves no slack to align the dynamic
+// shared memory by hand: its base is declared 1024-byte aligned, and a kernel
+// that finds it otherwise records FA_ERR_LAUNCH and returns.
+//
+// Hand-offs per query tile i (mbarriers; every wait bounded):
+//   q_full/q_empty[2], do_full/do_empty   producer <-> MMA (TMA ring slots)
+//   s_full   S^T(i) in TMEM          s_free   S^T(i) read: S^T(i+1) may be issued
+//   dp_full  dP^T(i) in TMEM         p_full   P^T(i) in shared memory
+//   p_free   dV(i) done: the P^T tile may take P^T(i+1)
+//   ds_full  dS^T(i) in shared memory (dP^T(i) has been read)
+//   ds_free  dK(i) and dQ(i) done: the dS^T tile may take dS^T(i+1)
+//   dq_full  dQ(i) in TMEM           dq_free  dQ(i) read: dP^T(i+1) may be issued
+// MMA order per i: S^T(i+1), dV(i), dK(i), dQ(i), dP^T(i+1).
+struct Bwd128Cfg {
+  static constexpr int D = 128;
+  static constexpr int BR = 128;
+  static constexpr int kTile = 128 * 128 * 2;       // K, V, Q, dO, P^T/dS^T tiles (32 KB)
+  static constexpr int kRegion = 128 * 128;         // 64-column block of a tile
+  static constexpr int kVecBytes = 2 * BR * 4;      // -LSE log2 e and D of one query tile
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kTile;
+  static constexpr int kOffQ = kOffV + kTile;       // two slots
+  static constexpr int kOffVec = kOffQ + 2 * kTile; // two slots
+  static constexpr int kOffDO = kOffVec + 2 * kVecBytes;
+  static constexpr int kOffP = kOffDO + kTile;
+  static constexpr int kOffDS = kOffP + kTile;
+  static constexpr int kOffBar = kOffDS + kTile;
+  // kv_full, q_full[2], q_empty[2], do_full, do_empty, s_full, s_free, dp_full, p_full,
+  // p_free, ds_full, ds_free, dq_full, dq_free, mma_done
+  static constexpr int kNumBars = 18;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16;
+  static_assert(kOffDO % 1024 == 0 && kOffP % 1024 == 0 && kOffDS % 1024 == 0,
+                "swizzled tiles need 1024-byte alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static constexpr int kColS = 0, kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 384;
+};
+// Register split for this kernel: 128 x (80 + 2 x 160 + 112) = 65536.
+constexpr int kB128RegsControl = 80;
+constexpr int kB128RegsSoftmax = 160;
+constexpr int kB128RegsDq = 112;
+static_assert(128 * (kB128RegsControl + 2 * kB128RegsSoftmax + kB128RegsDq) <= kBwdThreads * kBwdRegsLaunch,
+              "register split");
+
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_main_d128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                         const BwdParams p) {
+  using C = Bwd128Cfg;
+  constexpr int D = C::D;
+  constexpr int BR = C::BR;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {  // uniform across the CTA: nothing has started yet
+    if (threadIdx.x == 0) record_error(p.status, FA_ERR_LAUNCH);
+    return;
+  }
+  uint8_t* smem = smem_raw;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = bars + 3;
+  uint64_t* do_full = bars + 5;
+  uint64_t* do_empty = bars + 6;
+  uint64_t* s_full = bars + 7;
+  uint64_t* s_free = bars + 8;
+  uint64_t* dp_full = bars + 9;
+  uint64_t* p_full = bars + 10;
+  uint64_t* p_free = bars + 11;
+  uint64_t* ds_full = bars + 12;
+  uint64_t* ds_free = bars + 13;
+  uint64_t* dq_full = bars + 14;
+  uint64_t* dq_free = bars + 15;
+  uint64_t* mma_done = bars + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Work unit: (batch, kv head, key tile), key tile 0 first.
+  const int n_kt = (p.N + kTileN - 1) / kTileN;
+  const int kt = blockIdx.x % n_kt;
+  const int bkv = blockIdx.x / n_kt;
+  const int b = bkv / p.Hkv;
+  const int kvh = bkv % p.Hkv;
+  const int g = p.Hq / p.Hkv;
+  const int j0 = kt * kTileN;
+  const int n_qt = (p.N + BR - 1) / BR;
+  const int qt_first = p.causal ? j0 / BR : 0;
+  const int per_head = n_qt - qt_first;
+  const int n_it = g * per_head;
+  const float c = p.scale_log2;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1 + 32);
+      mbar_init(&q_empty[s], 1);
+    }
+    mbar_init(do_full, 1);
+    mbar_init(do_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 256);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 256);
+    mbar_init(p_free, 1);
+    mbar_init(ds_full, 256);
+    mbar_init(ds_free, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx w{abort_flag, p.status, p.wait_budget_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    regs_dec<kB128RegsControl, kBwdRegsLaunch>();
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(kv_full, 2 * C::kTile);
+#pragma unroll
+      for (int z = 0; z < 2; ++z) {
+        tma_load_3d(smem + C::kOffK + z * C::kRegion, &tmK, kv_full, z * 64, j0, bkv);
+        tma_load_3d(smem + C::kOffV + z * C::kRegion, &tmV, kv_full, z * 64, j0, bkv);
+      }
+    }
+    // Q_i (with its row vectors) as soon as its slot is free, then dO_i once dO_{i-1}
+    // has been used: Q runs up to two tiles ahead of dO.
+    bool ok = true;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int s = it & 1;
+      const int h = kvh * g + it / per_head;
+      const int i0 = (qt_first + it % per_head) * BR;
+      const int q_head = b * p.Hq + h;
+      if (!(ok = mbar_wait_spin(&q_empty[s], ((it >> 1) & 1) ^ 1, w))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&q_full[s], C::kTile);
+#pragma unroll
+        for (int z = 0; z < 2; ++z)
+          tma_load_3d(smem + C::kOffQ + s * C::kTile + z * C::kRegion, &tmQ, &q_full[s], z * 64, i0, q_head);
+      }
+      float* lse2 = reinterpret_cast<float*>(smem + C::kOffVec + s * C::kVecBytes);
+      float* dl = lse2 + BR;
+      const size_t rbase = (size_t)q_head * p.N;
+#pragma unroll
+      for (int r = lane; r < BR; r += 32) {
+        const int i = i0 + r;
+        const bool in = i < p.N;
+        lse2[r] = in ? -p.lse[rbase + i] * 1.4426950408889634f : -INFINITY;  // -LSE log2(e)
+        dl[r] = in ? p.delta[rbase + i] : 0.f;
+      }
+      mbar_arrive(&q_full[s]);
+      if (!(ok = mbar_wait_spin(do_empty, (it & 1) ^ 1, w))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(do_full, C::kTile);
+#pragma unroll
+        for (int z = 0; z < 2; ++z)
+          tma_load_3d(smem + C::kOffDO + z * C::kRegion, &tmDO, do_full, z * 64, i0, q_head);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    regs_dec<kB128RegsControl, kBwdRegsLaunch>();
+    const bool leader = lane == 0;
+    constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T: A, B K-major
+    constexpr uint32_t kIdKV = idesc_bf16_f32(128, 128, false, true);  // dV, dK: B MN-major
+    constexpr uint32_t kIdQ = idesc_bf16_f32(128, 128, true, true);    // dQ: A, B MN-major
+    const uint64_t dK_k = sdesc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
+    const uint64_t dV_k = sdesc_sw128(smem_u32(smem + C::kOffV), 16, 1024);
+    const uint64_t dK_mn = sdesc_sw128(smem_u32(smem + C::kOffK), C::kRegion, 1024);
+    const uint64_t dQ_k = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+    const uint64_t dQ_mn = sdesc_sw128(smem_u32(smem + C::kOffQ), C::kRegion, 1024);
+    const uint64_t dDO_k = sdesc_sw128(smem_u32(smem + C::kOffDO), 16, 1024);
+    const uint64_t dDO_mn = sdesc_sw128(smem_u32(smem + C::kOffDO), C::kRegion, 1024);
+    const uint64_t dP_k = sdesc_sw128(smem_u32(smem + C::kOffP), 16, 1024);
+    const uint64_t dS_k = sdesc_sw128(smem_u32(smem + C::kOffDS), 16, 1024);
+    const uint64_t dS_mn = sdesc_sw128(smem_u32(smem + C::kOffDS), C::kRegion, 1024);
+    // X^T = A B^T over the head dim (A = K or V, B = Q_i or dO_i, both K-major)
+    auto mma_scores = [&](uint64_t a0, uint64_t b0, uint32_t col) {
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * C::kRegion + (k & 3) * 32;
+        if (leader) mma_bf16_ss(tmem + col, desc_advance(a0, off), desc_advance(b0, off), kIdS, k > 0 ? 1u : 0u);
+      }
+    };
+    // acc += A B over the query rows (A = P^T or dS^T, K-major; B = dO_i or Q_i, MN-major)
+    auto mma_accum = [&](uint64_t a0, uint64_t b0, uint32_t col, bool first) {
+#pragma unroll
+      for (int k = 0; k < BR / 16; ++k) {
+        const uint32_t ao = (k >> 2) * C::kRegion + (k & 3) * 32;
+        if (leader)
+          mma_bf16_ss(tmem + col, desc_advance(a0, ao), desc_advance(b0, k * 2048), kIdKV,
+                      (!first || k > 0) ? 1u : 0u);
+      }
+    };
+    // dQ_i^T = K^T dS^T over the 128 keys (A = K^T: MN-major view of K; B = dS^T, MN-major):
+    // head-dim columns in TMEM lanes, so each warp's reduction of one query row is
+    // one coalesced 128-byte access.
+    auto mma_dq = [&]() {
+#pragma unroll
+      for (int k = 0; k < kTileN / 16; ++k)
+        if (leader)
+          mma_bf16_ss(tmem + C::kColDQ, desc_advance(dK_mn, k * 2048), desc_advance(dS_mn, k * 2048), kIdQ,
+                      k > 0 ? 1u : 0u);
+    };
+    bool ok = mbar_wait_spin(kv_full, 0, w);
+    if (ok && n_it > 0) ok = mbar_wait_spin(&q_full[0], 0, w);
+    if (ok && n_it > 0) ok = mbar_wait_spin(do_full, 0, w);
+    tc_fence_after();
+    if (ok && n_it > 0) {
+      mma_scores(dK_k, dQ_k, C::kColS);
+      if (leader) mma_commit(s_full);
+      mma_scores(dV_k, dDO_k, C::kColDP);
+      if (leader) mma_commit(dp_full);
+    }
+    for (int it = 0; it < n_it && ok; ++it) {
+      const uint32_t ph = it & 1;
+      const int s = it & 1;
+      // S^T(i+1) as soon as S^T(i) has been read
+      if (it + 1 < n_it) {
+        if (!(ok = mbar_wait_spin(&q_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
+        if (!(ok = mbar_wait_spin(s_free, ph, w))) break;
+        tc_fence_after();
+        mma_scores(dK_k, desc_advance(dQ_k, (s ^ 1) * C::kTile), C::kColS);
+        if (leader) mma_commit(s_full);
+      }
+      // dV += P^T dO_i
+      if (!(ok = mbar_wait_spin(p_full, ph, w))) break;
+      tc_fence_after();
+      mma_accum(dP_k, dDO_mn, C::kColDV, it == 0);
+      if (leader) {
+        mma_commit(p_free);
+        mma_commit(do_empty);
+      }
+      // dK += dS^T Q_i, then dQ_i = dS K into the dP^T columns (already read)
+      if (!(ok = mbar_wait_spin(ds_full, ph, w))) break;
+      tc_fence_after();
+      mma_accum(dS_k, desc_advance(dQ_mn, s * C::kTile), C::kColDK, it == 0);
+      if (leader) mma_commit(&q_empty[s]);
+      mma_dq();
+      if (leader) {
+        mma_commit(dq_full);
+        mma_commit(ds_free);
+      }
+      // dP^T(i+1) once dQ_i has been read out of TMEM
+      if (it + 1 < n_it) {
+        if (!(ok = mbar_wait_spin(dq_free, ph, w))) break;
+        if (!(ok = mbar_wait_spin(do_full, (it + 1) & 1, w))) break;
+        tc_fence_after();
+        mma_scores(dV_k, dDO_k, C::kColDP);
+        if (leader) mma_commit(dp_full);
+      }
+    }
+    if (leader) mma_commit(mma_done);
+    __syncwarp();
+    WaitCtx drain{abort_flag, p.status, 20000000ull};
+    volatile int zero = 0;
+    drain.abort_flag = &zero;
+    mbar_wait(mma_done, 0, drain);
+  } else if (warp < 4) {
+    regs_dec<kB128RegsControl, kBwdRegsLaunch>();
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ P^T and dS^T, 64 query columns each
+    regs_inc<kB128RegsSoftmax, kBwdRegsLaunch>();
+    constexpr int HB = 64;
+    const int half = (warp - 4) >> 2;
+    const int col0 = half * HB;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // key row within the tile
+    const int key = j0 + row;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t p_tile = smem_u32(smem + C::kOffP) + half * C::kRegion;
+    const uint32_t ds_tile = smem_u32(smem + C::kOffDS) + half * C::kRegion;
+    const bool key_valid = key < p.N;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it & 1;
+      const uint32_t ph = it & 1;
+      const int i0 = (qt_first + it % per_head) * BR + col0;  // first query of this half
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::kOffVec + s * C::kVecBytes) + col0;
+      const float* dl = lse2 + BR;
+      if (!mbar_wait_ns(&q_full[s], (it >> 1) & 1, w, kConsumerPollNs)) break;
+      if (!mbar_wait_ns(s_full, ph, w, kConsumerPollNs)) break;
+      tc_fence_after();
+      float pr[HB];
+#pragma unroll
+      for (int cc = 0; cc < HB / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + C::kColS + col0 + cc * 32, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pr[cc * 32 + i] = __uint_as_float(r[i]);
+      }
+      tc_fence_before();
+      mbar_arrive(s_free);
+      // P^T[key][q] = 2^(S c - LSE_q log2 e), zero for future queries and invalid keys.
+      const uint64_t c2 = f2_pack(c, c);
+      const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2);
+#pragma unroll
+      for (int i = 0; i < HB; i += 2) {
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(pr[i], pr[i + 1]), c2, nl2[i / 2]), x0, x1);
+        pr[i] = ex2(x0);
+        pr[i + 1] = ex2(x1);
+      }
+      if (p.causal && i0 < j0 + kTileN) {  // the diagonal tile only
+#pragma unroll
+        for (int i = 0; i < HB; ++i)
+          if (i0 + i < key) pr[i] = 0.f;
+      }
+      if (!key_valid) {
+#pragma unroll
+        for (int i = 0; i < HB; ++i) pr[i] = 0.f;
+      }
+      // the P^T tile is free once dV of the previous query tile is done
+      if (it >= 1 && !mbar_wait_ns(p_free, ph ^ 1, w, kConsumerPollNs)) break;
+#pragma unroll
+      for (int ch = 0; ch < HB / 8; ++ch) {
+        const int c0 = ch * 8;
+        st_shared_v4(p_tile + sw128_offset(row, ch), pack_bf16x2(pr[c0], pr[c0 + 1]),
+                     pack_bf16x2(pr[c0 + 2], pr[c0 + 3]), pack_bf16x2(pr[c0 + 4], pr[c0 + 5]),
+                     pack_bf16x2(pr[c0 + 6], pr[c0 + 7]));
+      }
+      fence_async_smem();
+      mbar_arrive(p_full);
+      // dS^T = P^T o (dP^T - D_q), 32 columns at a time
+      if (!mbar_wait_ns(dp_full, ph, w, kConsumerPollNs)) break;
+      tc_fence_after();
+      uint32_t dsp[HB / 2];
+      const uint64_t* dl2 = reinterpret_cast<const uint64_t*>(dl);
+#pragma unroll
+      for (int cc = 0; cc < HB / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + C::kColDP + col0 + cc * 32, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int q = cc * 32 + i;
+          float a, bb;
+          f2_unpack(f2_mul(f2_pack(pr[q], pr[q + 1]),
+                           f2_sub(f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), dl2[q / 2])),
+                    a, bb);
+          dsp[q / 2] = pack_bf16x2(a, bb);
+        }
+      }
+      // the dS^T tile is free once dK and dQ of the previous query tile are done
+      if (it >= 1 && !mbar_wait_ns(ds_free, ph ^ 1, w, kConsumerPollNs)) break;
+#pragma unroll
+      for (int ch = 0; ch < HB / 8; ++ch)
+        st_shared_v4(ds_tile + sw128_offset(row, ch), dsp[ch * 4], dsp[ch * 4 + 1], dsp[ch * 4 + 2],
+                     dsp[ch * 4 + 3]);
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+  } else {
+    // ------------------------------------------------------------ dQ reductions, dK / dV epilogue
+    regs_dec<kB128RegsDq, kBwdRegsLaunch>();
+    const int quarter = warp & 3;
+    const int tl = quarter * 32 + lane;  // TMEM lane
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int h = kvh * g + it / per_head;
+      const int i0 = (qt_first + it % per_head) * BR;
+      // lane = head-dim column, TMEM columns = the 128 query rows
+      float* base = p.dq_acc + ((size_t)(b * p.Hq + h) * p.N + i0) * D + tl;
+      const int nq = min(BR, p.N - i0);
+      if (!(ok = mbar_wait_ns(dq_full, it & 1, w, kConsumerPollNs))) break;
+      tc_fence_after();
+      auto reduce32 = [&](const uint32_t (&r)[32], int q0) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          if (q0 + q < nq) red_add(base + (size_t)(q0 + q) * D, __uint_as_float(r[q]));
+      };
+      // four 32-column loads, two buffers; dq_free as soon as the last one has landed
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tmem + lane_off + C::kColDQ, ra);
+      tmem_ld32(tmem + lane_off + C::kColDQ + 32, rb);
+      tmem_ld_wait(ra);
+      tmem_ld_wait(rb);
+      reduce32(ra, 0);
+      tmem_ld32(tmem + lane_off + C::kColDQ + 64, ra);
+      reduce32(rb, 32);
+      tmem_ld32(tmem + lane_off + C::kColDQ + 96, rb);
+      tmem_ld_wait(ra);
+      tmem_ld_wait(rb);
+      tc_fence_before();
+      mbar_arrive(dq_free);
+      reduce32(ra, 64);
+      reduce32(rb, 96);
+    }
+    if (ok && n_it > 0 && mbar_wait(mma_done, 0, w)) {
+      tc_fence_after();
+      // dK, dV rows: TMEM lane = key row
+      const int key = j0 + tl;
+      const bool valid = key < p.N;
+      const size_t row_idx = (size_t)bkv * p.N + key;
+      uint4* dk_dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + row_idx * D);
+      uint4* dv_dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + row_idx * D);
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which ? C::kColDK : C::kColDV;
+        const float mul = which ? p.scale : 1.f;
+        uint4* dst = which ? dk_dst : dv_dst;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + col + cc * 32, r);
+          tmem_ld_wait(r);
+          if (valid) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const int i = v4 * 8;
+              uint4 u;
+              u.x = pack_bf16x2(__uint_as_float(r[i]) * mul, __uint_as_float(r[i + 1]) * mul);
+              u.y = pack_bf16x2(__uint_as_float(r[i + 2]) * mul, __uint_as_float(r[i + 3]) * mul);
+              u.z = pack_bf16x2(__uint_as_float(r[i + 4]) * mul, __uint_as_float(r[i + 5]) * mul);
+              u.w = pack_bf16x2(__uint_as_float(r[i + 6]) * mul, __uint_as_float(r[i + 7]) * mul);
+              dst[cc * 4 + v4] = u;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 int sm_count() {
   static int n = 0;
   if (n == 0) {
@@ -594,6 +1056,15 @@ cudaError_t launch_preprocess_d(const BwdParams& p, cudaStream_t s) {
 template <int D>
 cudaError_t launch_main_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                           const BwdParams& p, cudaStream_t s) {
+  if (D == 128 && kBwd128Rows) {
+    using C = Bwd128Cfg;
+    cudaError_t e =
+        cudaFuncSetAttribute(bwd_main_d128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const long long grid = (long long)p.B * p.Hkv * ((p.N + kTileN - 1) / kTileN);
+    bwd_main_d128_kernel<<<(unsigned)grid, kBwdThreads, C::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
+    return cudaGetLastError();
+  }
   using C = BwdCfg<D>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
   cudaError_t e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -604,6 +1075,8 @@ cudaError_t launch_main_d(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 }
 
 }  // namespace
+
+int bwd_query_rows(int d) { return d == 128 ? (kBwd128Rows ? 128 : 64) : 128; }
 
 cudaError_t launch_bwd_preprocess(const BwdParams& p, cudaStream_t s) {
   return p.d == 128 ? launch_preprocess_d<128>(p, s) : launch_preprocess_d<64>(p, s);

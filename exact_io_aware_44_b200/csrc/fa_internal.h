@@ -52,6 +52,8 @@ cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const 
 cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, cudaStream_t s);
 cudaError_t launch_fwd_f32(const FwdF32Params& p, cudaStream_t s);
+// Query rows per tile of the main backward kernel for head dim d (its TMA box height).
+int bwd_query_rows(int d);
 // Backward phases: D and zeroed dQ accumulator; main kernel; dQ conversion.
 cudaError_t launch_bwd_preprocess(const BwdParams& p, cudaStream_t s);
 cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
