@@ -55,6 +55,12 @@ constexpr int kBwdThreads = 512;
 #endif
 // d = 128: 128-row query tiles (bwd_main_d128_kernel) instead of 64-row ones.
 constexpr bool kBwd128Rows = FA_BWD128_ROWS128 != 0;
+#ifndef FA_BWD_POLY_PAIRS
+#define FA_BWD_POLY_PAIRS 0
+#endif
+// Of every 8 pairs of P^T values, how many take 2^x by polynomial on the FMA pipe
+// instead of the SFU (128-row kernel).
+constexpr int kBwdPolyPairs = FA_BWD_POLY_PAIRS;
 // Register split: the launch gives 128 per thread (512 x 128 = 65536). The
 // control and dQ warpgroups lower to 96 and the two P/dS warpgroups raise to
 // 160: 128 x (96 + 2 x 160 + 96) = 65536.
@@ -581,44 +587,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // ---------------------------------------------------------------------------
 // With 128 query rows per tile every MMA has M = N = 128 (an N = 64 MMA runs at
 // about half the rate). Tensor Memory then holds exactly S^T [0,128),
-// dP^T [128,256), dV [256,384) and dK [384,512); the dQ tile of query tile i
-// (dQ^T = K^T dS^T, head-dim columns in TMEM lanes) reuses the dP^T columns once dP^T(i) has
-// been read, and dP^T(i+1) is issued once dQ(i) has been read. Shared memory
-// (226 KB): K, V, two Q slots (with -LSE log2 e and D per row), one dO slot, and
-// the P^T and dS^T tiles. The budget leaves no slack to align the dynamic
-// shared memory by hand: its base is declared 1024-byte aligned, and a kernel
-// that finds it otherwise records FA_ERR_LAUNCH and returns.
+// dP^T [128,256), dV [256,384) and dK [384,512):
+//   * P^T(i) is written back as bf16 over the S^T columns it came from (each
+//     warpgroup over the first half of its own 64 columns) and dV += P^T dO_i
+//     reads it from there, so P^T never goes through shared memory; S^T(i+1) is
+//     issued after dV(i).
+//   * dQ_i^T = K^T dS^T (head-dim columns in TMEM lanes, so each warp's fp32
+//     reduction of one query row is one coalesced 128-byte access) reuses the
+//     dP^T columns once dP^T(i) has been read, and dP^T(i+1) waits until dQ_i has
+//     been read out.
+// Shared memory (226 KB): K, V, two Q slots, two dO slots, the dS^T tile and the
+// per-row -LSE log2 e and D of the two Q slots. That leaves no slack to align the
+// base by hand, so it is declared 1024-byte aligned and checked at entry.
 //
 // Hand-offs per query tile i (mbarriers; every wait bounded):
-//   q_full/q_empty[2], do_full/do_empty   producer <-> MMA (TMA ring slots)
-//   s_full   S^T(i) in TMEM          s_free   S^T(i) read: S^T(i+1) may be issued
-//   dp_full  dP^T(i) in TMEM         p_full   P^T(i) in shared memory
-//   p_free   dV(i) done: the P^T tile may take P^T(i+1)
-//   ds_full  dS^T(i) in shared memory (dP^T(i) has been read)
-//   ds_free  dK(i) and dQ(i) done: the dS^T tile may take dS^T(i+1)
+//   q_full/q_empty[2], do_full/do_empty[2]   producer <-> MMA (TMA slots)
+//   s_full   S^T(i) in TMEM          p_full   P^T(i) in TMEM (S^T(i) has been read)
+//   dp_full  dP^T(i) in TMEM         ds_full  dS^T(i) in shared memory (dP^T(i) read)
+//   ds_free  dQ(i) and dK(i) done: the dS^T tile may take dS^T(i+1)
 //   dq_full  dQ(i) in TMEM           dq_free  dQ(i) read: dP^T(i+1) may be issued
-// MMA order per i: S^T(i+1), dV(i), dK(i), dQ(i), dP^T(i+1).
+// MMA order per i: dV(i), S^T(i+1), dQ(i), dK(i), dP^T(i+1).
 struct Bwd128Cfg {
   static constexpr int D = 128;
   static constexpr int BR = 128;
-  static constexpr int kTile = 128 * 128 * 2;       // K, V, Q, dO, P^T/dS^T tiles (32 KB)
+  static constexpr int kTile = 128 * 128 * 2;       // K, V, Q, dO, dS^T tiles (32 KB)
   static constexpr int kRegion = 128 * 128;         // 64-column block of a tile
   static constexpr int kVecBytes = 2 * BR * 4;      // -LSE log2 e and D of one query tile
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTile;
   static constexpr int kOffQ = kOffV + kTile;       // two slots
-  static constexpr int kOffVec = kOffQ + 2 * kTile; // two slots
-  static constexpr int kOffDO = kOffVec + 2 * kVecBytes;
-  static constexpr int kOffP = kOffDO + kTile;
-  static constexpr int kOffDS = kOffP + kTile;
-  static constexpr int kOffBar = kOffDS + kTile;
-  // kv_full, q_full[2], q_empty[2], do_full, do_empty, s_full, s_free, dp_full, p_full,
-  // p_free, ds_full, ds_free, dq_full, dq_free, mma_done
-  static constexpr int kNumBars = 18;
+  static constexpr int kOffDO = kOffQ + 2 * kTile;  // two slots
+  static constexpr int kOffDS = kOffDO + 2 * kTile;
+  static constexpr int kOffVec = kOffDS + kTile;    // two slots
+  static constexpr int kOffBar = kOffVec + 2 * kVecBytes;
+  // kv_full, q_full[2], q_empty[2], do_full[2], do_empty[2], s_full, p_full, dp_full,
+  // ds_full, ds_free, dq_full, dq_free, mma_done
+  static constexpr int kNumBars = 17;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
-  static_assert(kOffDO % 1024 == 0 && kOffP % 1024 == 0 && kOffDS % 1024 == 0,
-                "swizzled tiles need 1024-byte alignment");
+  static_assert(kOffDS % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static constexpr int kColS = 0, kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 384;
 };
@@ -647,12 +654,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* q_full = bars + 1;
   uint64_t* q_empty = bars + 3;
   uint64_t* do_full = bars + 5;
-  uint64_t* do_empty = bars + 6;
-  uint64_t* s_full = bars + 7;
-  uint64_t* s_free = bars + 8;
-  uint64_t* dp_full = bars + 9;
+  uint64_t* do_empty = bars + 7;
+  uint64_t* s_full = bars + 9;
   uint64_t* p_full = bars + 10;
-  uint64_t* p_free = bars + 11;
+  uint64_t* dp_full = bars + 11;
   uint64_t* ds_full = bars + 12;
   uint64_t* ds_free = bars + 13;
   uint64_t* dq_full = bars + 14;
@@ -683,14 +688,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&q_full[s], 1 + 32);
       mbar_init(&q_empty[s], 1);
+      mbar_init(&do_full[s], 1);
+      mbar_init(&do_empty[s], 1);
     }
-    mbar_init(do_full, 1);
-    mbar_init(do_empty, 1);
     mbar_init(s_full, 1);
-    mbar_init(s_free, 256);
-    mbar_init(dp_full, 1);
     mbar_init(p_full, 256);
-    mbar_init(p_free, 1);
+    mbar_init(dp_full, 1);
     mbar_init(ds_full, 256);
     mbar_init(ds_free, 1);
     mbar_init(dq_full, 1);
@@ -724,15 +727,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_3d(smem + C::kOffV + z * C::kRegion, &tmV, kv_full, z * 64, j0, bkv);
       }
     }
-    // Q_i (with its row vectors) as soon as its slot is free, then dO_i once dO_{i-1}
-    // has been used: Q runs up to two tiles ahead of dO.
+    // Q_i (with its row vectors) and dO_i, each as soon as its slot is free.
     bool ok = true;
     for (int it = 0; it < n_it && ok; ++it) {
       const int s = it & 1;
+      const uint32_t use_par = ((it >> 1) & 1) ^ 1;  // parity of the slot's previous release
       const int h = kvh * g + it / per_head;
       const int i0 = (qt_first + it % per_head) * BR;
       const int q_head = b * p.Hq + h;
-      if (!(ok = mbar_wait_spin(&q_empty[s], ((it >> 1) & 1) ^ 1, w))) break;
+      if (!(ok = mbar_wait_spin(&q_empty[s], use_par, w))) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(&q_full[s], C::kTile);
 #pragma unroll
@@ -750,12 +753,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         dl[r] = in ? p.delta[rbase + i] : 0.f;
       }
       mbar_arrive(&q_full[s]);
-      if (!(ok = mbar_wait_spin(do_empty, (it & 1) ^ 1, w))) break;
+      if (!(ok = mbar_wait_spin(&do_empty[s], use_par, w))) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(do_full, C::kTile);
+        mbar_arrive_expect_tx(&do_full[s], C::kTile);
 #pragma unroll
         for (int z = 0; z < 2; ++z)
-          tma_load_3d(smem + C::kOffDO + z * C::kRegion, &tmDO, do_full, z * 64, i0, q_head);
+          tma_load_3d(smem + C::kOffDO + s * C::kTile + z * C::kRegion, &tmDO, &do_full[s], z * 64, i0, q_head);
       }
       __syncwarp();
     }
@@ -765,7 +768,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool leader = lane == 0;
     constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T: A, B K-major
     constexpr uint32_t kIdKV = idesc_bf16_f32(128, 128, false, true);  // dV, dK: B MN-major
-    constexpr uint32_t kIdQ = idesc_bf16_f32(128, 128, true, true);    // dQ: A, B MN-major
+    constexpr uint32_t kIdQ = idesc_bf16_f32(128, 128, true, true);    // dQ^T: A, B MN-major
     const uint64_t dK_k = sdesc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
     const uint64_t dV_k = sdesc_sw128(smem_u32(smem + C::kOffV), 16, 1024);
     const uint64_t dK_mn = sdesc_sw128(smem_u32(smem + C::kOffK), C::kRegion, 1024);
@@ -773,7 +776,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t dQ_mn = sdesc_sw128(smem_u32(smem + C::kOffQ), C::kRegion, 1024);
     const uint64_t dDO_k = sdesc_sw128(smem_u32(smem + C::kOffDO), 16, 1024);
     const uint64_t dDO_mn = sdesc_sw128(smem_u32(smem + C::kOffDO), C::kRegion, 1024);
-    const uint64_t dP_k = sdesc_sw128(smem_u32(smem + C::kOffP), 16, 1024);
     const uint64_t dS_k = sdesc_sw128(smem_u32(smem + C::kOffDS), 16, 1024);
     const uint64_t dS_mn = sdesc_sw128(smem_u32(smem + C::kOffDS), C::kRegion, 1024);
     // X^T = A B^T over the head dim (A = K or V, B = Q_i or dO_i, both K-major)
@@ -784,19 +786,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (leader) mma_bf16_ss(tmem + col, desc_advance(a0, off), desc_advance(b0, off), kIdS, k > 0 ? 1u : 0u);
       }
     };
-    // acc += A B over the query rows (A = P^T or dS^T, K-major; B = dO_i or Q_i, MN-major)
-    auto mma_accum = [&](uint64_t a0, uint64_t b0, uint32_t col, bool first) {
+    // dV += P^T dO_i: A = P^T in TMEM (query columns q: warpgroup q / 64's packed
+    // pairs at S^T columns 64 (q / 64) + (q % 64) / 2), B = dO_i (MN-major)
+    auto mma_dv = [&](uint64_t b0, bool first) {
+#pragma unroll
+      for (int k = 0; k < BR / 16; ++k) {
+        const uint32_t acol = C::kColS + (k >> 2) * 64 + (k & 3) * 8;
+        if (leader)
+          mma_bf16_ts(tmem + C::kColDV, tmem + acol, desc_advance(b0, k * 2048), kIdKV, (!first || k > 0) ? 1u : 0u);
+      }
+    };
+    // dK += dS^T Q_i (A = dS^T, K-major; B = Q_i, MN-major)
+    auto mma_dk = [&](uint64_t b0, bool first) {
 #pragma unroll
       for (int k = 0; k < BR / 16; ++k) {
         const uint32_t ao = (k >> 2) * C::kRegion + (k & 3) * 32;
         if (leader)
-          mma_bf16_ss(tmem + col, desc_advance(a0, ao), desc_advance(b0, k * 2048), kIdKV,
+          mma_bf16_ss(tmem + C::kColDK, desc_advance(dS_k, ao), desc_advance(b0, k * 2048), kIdKV,
                       (!first || k > 0) ? 1u : 0u);
       }
     };
-    // dQ_i^T = K^T dS^T over the 128 keys (A = K^T: MN-major view of K; B = dS^T, MN-major):
-    // head-dim columns in TMEM lanes, so each warp's reduction of one query row is
-    // one coalesced 128-byte access.
+    // dQ_i^T = K^T dS^T over the 128 keys (A = K^T: MN-major view of K; B = dS^T, MN-major)
     auto mma_dq = [&]() {
 #pragma unroll
       for (int k = 0; k < kTileN / 16; ++k)
@@ -806,7 +816,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     };
     bool ok = mbar_wait_spin(kv_full, 0, w);
     if (ok && n_it > 0) ok = mbar_wait_spin(&q_full[0], 0, w);
-    if (ok && n_it > 0) ok = mbar_wait_spin(do_full, 0, w);
+    if (ok && n_it > 0) ok = mbar_wait_spin(&do_full[0], 0, w);
     tc_fence_after();
     if (ok && n_it > 0) {
       mma_scores(dK_k, dQ_k, C::kColS);
@@ -817,38 +827,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int it = 0; it < n_it && ok; ++it) {
       const uint32_t ph = it & 1;
       const int s = it & 1;
-      // S^T(i+1) as soon as S^T(i) has been read
+      // dV += P^T dO_i, then S^T(i+1) into the columns P^T(i) came from (one
+      // thread's MMAs execute in issue order)
+      if (!(ok = mbar_wait_spin(p_full, ph, w))) break;
+      tc_fence_after();
+      mma_dv(desc_advance(dDO_mn, s * C::kTile), it == 0);
+      if (leader) mma_commit(&do_empty[s]);
       if (it + 1 < n_it) {
         if (!(ok = mbar_wait_spin(&q_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
-        if (!(ok = mbar_wait_spin(s_free, ph, w))) break;
         tc_fence_after();
         mma_scores(dK_k, desc_advance(dQ_k, (s ^ 1) * C::kTile), C::kColS);
         if (leader) mma_commit(s_full);
       }
-      // dV += P^T dO_i
-      if (!(ok = mbar_wait_spin(p_full, ph, w))) break;
-      tc_fence_after();
-      mma_accum(dP_k, dDO_mn, C::kColDV, it == 0);
-      if (leader) {
-        mma_commit(p_free);
-        mma_commit(do_empty);
-      }
-      // dK += dS^T Q_i, then dQ_i = dS K into the dP^T columns (already read)
+      // dQ_i into the dP^T columns (already read), then dK += dS^T Q_i
       if (!(ok = mbar_wait_spin(ds_full, ph, w))) break;
       tc_fence_after();
-      mma_accum(dS_k, desc_advance(dQ_mn, s * C::kTile), C::kColDK, it == 0);
-      if (leader) mma_commit(&q_empty[s]);
       mma_dq();
+      if (leader) mma_commit(dq_full);
+      mma_dk(desc_advance(dQ_mn, s * C::kTile), it == 0);
       if (leader) {
-        mma_commit(dq_full);
+        mma_commit(&q_empty[s]);
         mma_commit(ds_free);
       }
       // dP^T(i+1) once dQ_i has been read out of TMEM
       if (it + 1 < n_it) {
         if (!(ok = mbar_wait_spin(dq_free, ph, w))) break;
-        if (!(ok = mbar_wait_spin(do_full, (it + 1) & 1, w))) break;
+        if (!(ok = mbar_wait_spin(&do_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
         tc_fence_after();
-        mma_scores(dV_k, dDO_k, C::kColDP);
+        mma_scores(dV_k, desc_advance(dDO_k, (s ^ 1) * C::kTile), C::kColDP);
         if (leader) mma_commit(dp_full);
       }
     }
@@ -870,7 +876,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = quarter * 32 + lane;  // key row within the tile
     const int key = j0 + row;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t p_tile = smem_u32(smem + C::kOffP) + half * C::kRegion;
     const uint32_t ds_tile = smem_u32(smem + C::kOffDS) + half * C::kRegion;
     const bool key_valid = key < p.N;
     for (int it = 0; it < n_it; ++it) {
@@ -883,16 +888,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!mbar_wait_ns(s_full, ph, w, kConsumerPollNs)) break;
       tc_fence_after();
       float pr[HB];
+      {
+        uint32_t r0[32], r1[32];  // both loads in flight before the one wait
+        tmem_ld32(tmem + lane_off + C::kColS + col0, r0);
+        tmem_ld32(tmem + lane_off + C::kColS + col0 + 32, r1);
+        tmem_ld_wait(r0);
+        tmem_ld_wait(r1);
 #pragma unroll
-      for (int cc = 0; cc < HB / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_off + C::kColS + col0 + cc * 32, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pr[cc * 32 + i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 32; ++i) {
+          pr[i] = __uint_as_float(r0[i]);
+          pr[32 + i] = __uint_as_float(r1[i]);
+        }
       }
-      tc_fence_before();
-      mbar_arrive(s_free);
       // P^T[key][q] = 2^(S c - LSE_q log2 e), zero for future queries and invalid keys.
       const uint64_t c2 = f2_pack(c, c);
       const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2);
@@ -900,8 +907,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int i = 0; i < HB; i += 2) {
         float x0, x1;
         f2_unpack(f2_fma(f2_pack(pr[i], pr[i + 1]), c2, nl2[i / 2]), x0, x1);
-        pr[i] = ex2(x0);
-        pr[i + 1] = ex2(x1);
+        if (((i / 2) & 7) < kBwdPolyPairs) {  // part of the exponentials on the FMA pipe
+          ex2_poly2(x0, x1, pr[i], pr[i + 1]);
+        } else {
+          pr[i] = ex2(x0);
+          pr[i + 1] = ex2(x1);
+        }
       }
       if (p.causal && i0 < j0 + kTileN) {  // the diagonal tile only
 #pragma unroll
@@ -912,16 +923,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int i = 0; i < HB; ++i) pr[i] = 0.f;
       }
-      // the P^T tile is free once dV of the previous query tile is done
-      if (it >= 1 && !mbar_wait_ns(p_free, ph ^ 1, w, kConsumerPollNs)) break;
+      // P^T as bf16 pairs over the first 32 of this warpgroup's S^T columns (read above)
+      {
+        uint32_t pk[32];
 #pragma unroll
-      for (int ch = 0; ch < HB / 8; ++ch) {
-        const int c0 = ch * 8;
-        st_shared_v4(p_tile + sw128_offset(row, ch), pack_bf16x2(pr[c0], pr[c0 + 1]),
-                     pack_bf16x2(pr[c0 + 2], pr[c0 + 3]), pack_bf16x2(pr[c0 + 4], pr[c0 + 5]),
-                     pack_bf16x2(pr[c0 + 6], pr[c0 + 7]));
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[2 * i], pr[2 * i + 1]);
+        tmem_st32(tmem + lane_off + C::kColS + col0, pk);
+        tmem_st_wait();
       }
-      fence_async_smem();
+      tc_fence_before();
       mbar_arrive(p_full);
       // dS^T = P^T o (dP^T - D_q), 32 columns at a time
       if (!mbar_wait_ns(dp_full, ph, w, kConsumerPollNs)) break;
@@ -943,7 +953,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           dsp[q / 2] = pack_bf16x2(a, bb);
         }
       }
-      // the dS^T tile is free once dK and dQ of the previous query tile are done
+      // the dS^T tile is free once dQ and dK of the previous query tile are done
       if (it >= 1 && !mbar_wait_ns(ds_free, ph ^ 1, w, kConsumerPollNs)) break;
 #pragma unroll
       for (int ch = 0; ch < HB / 8; ++ch)
@@ -973,22 +983,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int q = 0; q < 32; ++q)
           if (q0 + q < nq) red_add(base + (size_t)(q0 + q) * D, __uint_as_float(r[q]));
       };
-      // four 32-column loads, two buffers; dq_free as soon as the last one has landed
-      uint32_t ra[32], rb[32];
+      // four 32-column loads into three buffers; dq_free as soon as the last one has
+      // landed (only one chunk's reductions are issued before it: they queue behind
+      // the memory system and would hold up the next dP^T)
+      uint32_t ra[32], rb[32], rc[32];
       tmem_ld32(tmem + lane_off + C::kColDQ, ra);
       tmem_ld32(tmem + lane_off + C::kColDQ + 32, rb);
+      tmem_ld32(tmem + lane_off + C::kColDQ + 64, rc);
       tmem_ld_wait(ra);
       tmem_ld_wait(rb);
+      tmem_ld_wait(rc);
       reduce32(ra, 0);
-      tmem_ld32(tmem + lane_off + C::kColDQ + 64, ra);
-      reduce32(rb, 32);
-      tmem_ld32(tmem + lane_off + C::kColDQ + 96, rb);
+      tmem_ld32(tmem + lane_off + C::kColDQ + 96, ra);
       tmem_ld_wait(ra);
-      tmem_ld_wait(rb);
       tc_fence_before();
       mbar_arrive(dq_free);
-      reduce32(ra, 64);
-      reduce32(rb, 96);
+      reduce32(rb, 32);
+      reduce32(rc, 64);
+      reduce32(ra, 96);
     }
     if (ok && n_it > 0 && mbar_wait(mma_done, 0, w)) {
       tc_fence_after();
