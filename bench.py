@@ -47,17 +47,32 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 # source makes the figure stale and the bench reports null.
 NCU_TRAFFIC = {
     # profiles/bwd_main_d128_B2H32N8192_causal.md
-    ("bwd_main", "c3"): {"bytes_per_launch": 809782016 + 490684160, "csrc_sha": "cf77055da08ab318"},
+    ("bwd_main", "c3"): {"bytes_per_launch": 809986560 + 491049984, "csrc_sha": "7497d3bd4abc43c9"},
+}
+
+
+# The source text each kernel is built from: its own definition (start marker up
+# to end marker) plus the shared device helpers. Edits elsewhere in the file (the
+# other head-dim variant, comments) leave the recorded counters valid.
+KERNEL_SOURCES = {
+    "bwd_main": ("fa_bwd_sm100.cu", [("__device__ __forceinline__ void red_add_v4", "// ----"),
+                                     ("struct Bwd128Cfg {", "int sm_count() {")]),
+    "fwd": ("fa_fwd_sm100.cu", [("", None)]),
 }
 
 
 def kernel_source_hash(kernel: str) -> str:
-    fname = {"bwd_main": "fa_bwd_sm100.cu", "fwd": "fa_fwd_sm100.cu"}[kernel]
-    paths = [os.path.join(ROOT, "exact_io_aware_44_b200", "csrc", f) for f in (fname, "sm100.cuh")]
+    fname, spans = KERNEL_SOURCES[kernel]
+    csrc = os.path.join(ROOT, "exact_io_aware_44_b200", "csrc")
     h = hashlib.sha256()
-    for p in paths:
-        with open(p, "rb") as f:
-            h.update(f.read())
+    with open(os.path.join(csrc, fname)) as f:
+        text = f.read()
+    for start, end in spans:
+        a = text.index(start) if start else 0
+        b = text.index(end, a) if end else len(text)
+        h.update(text[a:b].encode())
+    with open(os.path.join(csrc, "sm100.cuh"), "rb") as f:
+        h.update(f.read())
     return h.hexdigest()[:16]
 
 

@@ -7,38 +7,29 @@
 // For L = sum(O o dO), with D_i = sum_c dO_ic O_ic and dS = P o (dP - D):
 //   dV = P^T dO,   dP = dO V^T,   dK = scale dS^T Q,   dQ = scale dS K.
 //
-// Three kernels:
+// Kernels:
 //   bwd_preprocess  D = rowsum(dO o O) (fp32) and zeroes the fp32 dQ accumulator.
 //   bwd_main        one CTA per 128-key tile of one (batch, kv head). It keeps K
 //                   and V in shared memory and dK, dV in Tensor Memory, and loops
-//                   over the query heads of its GQA group and the query tiles
-//                   that can see its keys. Per query tile i (BR rows):
+//                   over the query heads of its GQA group and the 128-row query
+//                   tiles that can see its keys. Per query tile i:
 //                     S^T = K Q_i^T, dP^T = V dO_i^T          (tcgen05.mma -> TMEM)
 //                     P^T = 2^(S^T c - LSE_i log2 e), dS^T = P^T o (dP^T - D_i)
 //                     dV += P^T dO_i, dK += dS^T Q_i            (TMEM accumulators)
-//                     dQ_i partial = dS K (d = 64) or K^T dS^T (d = 128) -> TMEM,
-//                     then added to the fp32 accumulator with red.global.add.
+//                     dQ_i partial -> TMEM, then added to the fp32 accumulator
+//                     with red.global.add.
+//                   Two variants, one per head dim: bwd_main_kernel<64> and
+//                   bwd_main_d128_kernel (described where each is defined).
 //   bwd_convert     dQ = bf16(scale * accumulator).
 //
 // bwd_main roles (512 threads):
 //   warp 0      producer: K, V once (TMA); per query tile Q_i, dO_i (TMA) and
-//               -LSE_i log2(e), D_i (plain loads) into a ring of stages.
+//               -LSE_i log2(e), D_i (plain loads) into shared-memory slots.
 //   warp 1      allocates TMEM; one lane issues every tcgen05.mma.
 //   warps 4-11  two warpgroups, thread = key row; warpgroup h computes P^T and
-//               dS^T for query columns [h BR/2, (h+1) BR/2) and writes them to
-//               shared memory in the 128-byte-swizzled K-major layout.
+//               dS^T for query columns [64 h, 64 h + 64).
 //   warps 12-15 thread = TMEM lane of the dQ tile: reads it and issues the fp32
 //               reductions; at the end, writes dK and dV.
-//
-// MMA issue order per query tile i: S(i+1), dV(i), dP(i+1), dK(i), dQ(i). The
-// next tile's scores are issued as soon as the current ones have been read out
-// of TMEM, and dP(i+1) as soon as dP(i) has, so they are computed while the
-// elementwise warpgroups still work on P(i) and dS(i).
-//
-// Query tiles are BR = 64 rows for d = 128 (so dQ^T = K^T dS^T has M = d = 128)
-// and BR = 128 rows for d = 64 (so dQ = dS K has M = 128 query rows). TMEM
-// columns: S^T [0, BR), dP^T [BR, 2BR), dQ [2BR, 2BR + 64), dV [512 - 2d, 512 - d),
-// dK [512 - d, 512).
 #include <math.h>
 
 #include <algorithm>
@@ -50,11 +41,6 @@ namespace fa {
 namespace {
 
 constexpr int kBwdThreads = 512;
-#ifndef FA_BWD128_ROWS128
-#define FA_BWD128_ROWS128 1
-#endif
-// d = 128: 128-row query tiles (bwd_main_d128_kernel) instead of 64-row ones.
-constexpr bool kBwd128Rows = FA_BWD128_ROWS128 != 0;
 #ifndef FA_BWD_POLY_PAIRS
 #define FA_BWD_POLY_PAIRS 0
 #endif
@@ -71,9 +57,19 @@ constexpr int kBwdRegsDq = 96;
 static_assert(128 * (kBwdRegsControl + 2 * kBwdRegsSoftmax + kBwdRegsDq) <= kBwdThreads * kBwdRegsLaunch,
               "register split");
 
+// ---------------------------------------------------------------------------
+// main backward kernel, d = 64
+// ---------------------------------------------------------------------------
+// Query tiles of BR = 128 rows; dQ = dS K has M = 128 query rows (TMEM lanes)
+// and N = d = 64. TMEM columns: S^T [0, 128), dP^T [128, 256), dQ [256, 320),
+// dV [384, 448), dK [448, 512). P^T and dS^T go through shared memory in the
+// 128-byte-swizzled K-major layout. MMA issue order per query tile i: S(i+1),
+// dV(i), dP(i+1), dK(i), dQ(i): the next tile's scores are issued as soon as the
+// current ones have been read out of TMEM, and dP(i+1) as soon as dP(i) has.
 template <int D>
 struct BwdCfg {
-  static constexpr int BR = (D == 128) ? 64 : 128;  // query rows per tile
+  static_assert(D == 64, "bwd_main_kernel serves d = 64; d = 128 has bwd_main_d128_kernel");
+  static constexpr int BR = 128;                    // query rows per tile
   static constexpr int kStages = 3;
   static constexpr int kKVBytes = kTileN * D * 2;   // K or V tile (128 keys)
   static constexpr int kKVRegion = kTileN * 128;    // 64-column block of a K/V tile
@@ -332,11 +328,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                       (!first || k > 0) ? 1u : 0u);
       }
     };
-    // dQ (d = 64): A = dS (MN-major view of dS^T), B = K (MN-major), over the 128 keys.
-    // dQ^T (d = 128): A = K^T (MN-major view of K), B = dS^T (MN-major), over the 128 keys.
+    // dQ = dS K: A = dS (MN-major view of dS^T), B = K (MN-major), over the 128 keys.
     auto mma_dq = [&]() {
-      const uint64_t a0 = (D == 128) ? dK_mn : dDs_mn;
-      const uint64_t b0 = (D == 128) ? dDs_mn : dK_mn;
+      const uint64_t a0 = dDs_mn;
+      const uint64_t b0 = dK_mn;
 #pragma unroll
       for (int k = 0; k < kTileN / 16; ++k)
         if (leader) mma_bf16_ss(tmem + C::kColDQ, desc_advance(a0, k * 2048), desc_advance(b0, k * 2048), kIdQ,
@@ -514,29 +509,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_ld_wait(r1);
       tc_fence_before();
       mbar_arrive(dq_free);
-      if (D == 128) {
-        // lane = head-dim column, TMEM columns = the BR = 64 query rows
-        float* base = p.dq_acc + (head_row0 + i0) * D + tl;
-        const int nq = min(64, p.N - i0);
+      // lane = query row, TMEM columns = the 64 head-dim columns
+      if (i0 + tl < p.N) {
+        float* base = p.dq_acc + (head_row0 + i0 + tl) * D;
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (q < nq) red_add(base + (size_t)q * D, __uint_as_float(r0[q]));
+        for (int v = 0; v < 8; ++v)
+          red_add_v4(base + v * 4, __uint_as_float(r0[v * 4]), __uint_as_float(r0[v * 4 + 1]),
+                     __uint_as_float(r0[v * 4 + 2]), __uint_as_float(r0[v * 4 + 3]));
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (q + 32 < nq) red_add(base + (size_t)(q + 32) * D, __uint_as_float(r1[q]));
-      } else {
-        // lane = query row, TMEM columns = the 64 head-dim columns
-        if (i0 + tl < p.N) {
-          float* base = p.dq_acc + (head_row0 + i0 + tl) * D;
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            red_add_v4(base + v * 4, __uint_as_float(r0[v * 4]), __uint_as_float(r0[v * 4 + 1]),
-                       __uint_as_float(r0[v * 4 + 2]), __uint_as_float(r0[v * 4 + 3]));
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            red_add_v4(base + 32 + v * 4, __uint_as_float(r1[v * 4]), __uint_as_float(r1[v * 4 + 1]),
-                       __uint_as_float(r1[v * 4 + 2]), __uint_as_float(r1[v * 4 + 3]));
-        }
+        for (int v = 0; v < 8; ++v)
+          red_add_v4(base + 32 + v * 4, __uint_as_float(r1[v * 4]), __uint_as_float(r1[v * 4 + 1]),
+                     __uint_as_float(r1[v * 4 + 2]), __uint_as_float(r1[v * 4 + 3]));
       }
     }
     if (ok && n_it > 0 && mbar_wait(mma_done, 0, w)) {
@@ -1068,27 +1051,27 @@ cudaError_t launch_preprocess_d(const BwdParams& p, cudaStream_t s) {
 template <int D>
 cudaError_t launch_main_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                           const BwdParams& p, cudaStream_t s) {
-  if (D == 128 && kBwd128Rows) {
+  const long long grid = (long long)p.B * p.Hkv * ((p.N + kTileN - 1) / kTileN);
+  if constexpr (D == 128) {
     using C = Bwd128Cfg;
     cudaError_t e =
         cudaFuncSetAttribute(bwd_main_d128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const long long grid = (long long)p.B * p.Hkv * ((p.N + kTileN - 1) / kTileN);
     bwd_main_d128_kernel<<<(unsigned)grid, kBwdThreads, C::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
-    return cudaGetLastError();
+  } else {
+    using C = BwdCfg<D>;
+    static_assert(C::kSmemBytes <= 232448, "shared memory budget");
+    cudaError_t e =
+        cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    bwd_main_kernel<D><<<(unsigned)grid, kBwdThreads, C::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
   }
-  using C = BwdCfg<D>;
-  static_assert(C::kSmemBytes <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  const long long grid = (long long)p.B * p.Hkv * ((p.N + kTileN - 1) / kTileN);
-  bwd_main_kernel<D><<<(unsigned)grid, kBwdThreads, C::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-int bwd_query_rows(int d) { return d == 128 ? (kBwd128Rows ? 128 : 64) : 128; }
+int bwd_query_rows(int) { return 128; }
 
 cudaError_t launch_bwd_preprocess(const BwdParams& p, cudaStream_t s) {
   return p.d == 128 ? launch_preprocess_d<128>(p, s) : launch_preprocess_d<64>(p, s);
