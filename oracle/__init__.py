@@ -14,6 +14,10 @@ Parity status per function (what pins it; see tests/test_oracle.py):
                           pinned: equal the full oracle restricted to the sampled rows.
   head_probs64            pinned: SciPy softmax of brute-force scores, zero above the
                           causal diagonal, P V reproduces the brute-force output.
+  decode_fwd64            pinned: pure-Python brute force (decode_naive_loops), equals
+                          attention_fwd64 when Nq = Nk, equals the last rows of the square
+                          causal attention when the queries are the sequence's last rows,
+                          and a single causal query sees every key.
   finite_diff_grads64     pinned: exact gradients of closed-form cases.
 The pages print no worked numeric example, so no value is pinned to a printed number.
 """
@@ -22,6 +26,8 @@ from .attention64 import (  # noqa: F401
     attention_bwd64,
     attention_fwd64,
     attention_naive_loops,
+    decode_fwd64,
+    decode_naive_loops,
     finite_diff_grads64,
     group_bwd_sampled64,
     head_fwd64,

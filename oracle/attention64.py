@@ -117,6 +117,52 @@ def attention_fwd64(q, k, v, causal, scale=None):
     return o, lse
 
 
+def decode_fwd64(q, k, v, causal, scale=None):
+    """Attention of Nq new queries against a cache of Nk >= Nq keys (decode).
+
+    q [B, Hq, Nq, d]; k, v [B, Hkv, Nk, d] -> O [B, Hq, Nq, d], LSE [B, Hq, Nq].
+    The queries are the last Nq positions of the sequence: query i sits at
+    position Nk - Nq + i and, when causal, sees keys j <= Nk - Nq + i (with
+    Nq = Nk this is the square causal mask of attention_fwd64). One-pass softmax
+    over each full key row, as in head_fwd64.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    if causal and Nq > Nk:
+        raise ValueError("causal decode needs Nq <= Nk")
+    g = Hq // Hkv
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            s = scale * (q[b, h] @ k[b, h // g].T)          # [Nq, Nk]
+            if causal:
+                pos = Nk - Nq + np.arange(Nq)[:, None]
+                s = np.where(np.arange(Nk)[None, :] <= pos, s, -np.inf)
+            p, lse[b, h] = _softmax_rows(s)
+            o[b, h] = p @ v[b, h // g]
+    return o, lse
+
+
+def decode_naive_loops(q, k, v, causal, scale):
+    """Pure-Python brute force of decode_fwd64 for one head (lists of rows)."""
+    import math
+    nq, nk = len(q), len(k)
+    out, lses = [], []
+    for i in range(nq):
+        keys = range(nk - nq + i + 1) if causal else range(nk)
+        s = [scale * sum(a * b for a, b in zip(q[i], k[j])) for j in keys]
+        mx = max(s)
+        z = sum(math.exp(x - mx) for x in s)
+        out.append([sum(math.exp(s[t] - mx) / z * v[j][c] for t, j in enumerate(keys)) for c in range(len(v[0]))])
+        lses.append(mx + math.log(z))
+    return out, lses
+
+
 def _probs(q_rows, kh, lse_rows, scale, row0, causal):
     """P recomputed from Q, K and the saved LSE (the backward's recomputation)."""
     s = _scores(q_rows, kh, scale, row0, causal)

@@ -297,6 +297,37 @@ def test_head_probs_are_the_softmax_of_brute_force_scores():
         np.testing.assert_allclose(p @ v, np.array(o_ref)[sel], rtol=1e-10, atol=1e-12)
 
 
+def test_decode_oracle_pins():
+    scale = 0.35
+    # brute force on tiny shapes, GQA, causal and not
+    for causal in (True, False):
+        for (Nq, Nk) in ((1, 1), (1, 5), (3, 7), (4, 4)):
+            q, k, v = rand((1, 4, Nq, 3), 51), rand((1, 2, Nk, 3), 52), rand((1, 2, Nk, 3), 53)
+            o, lse = oracle.decode_fwd64(q, k, v, causal, scale)
+            for h in range(4):
+                ob, lb = oracle.decode_naive_loops(q[0, h].tolist(), k[0, h // 2].tolist(), v[0, h // 2].tolist(),
+                                                    causal, scale)
+                np.testing.assert_allclose(o[0, h], np.array(ob), rtol=1e-12, atol=1e-12)
+                np.testing.assert_allclose(lse[0, h], np.array(lb), rtol=1e-12, atol=1e-12)
+    # Nq = Nk is the square attention; the last Nq rows of a causal sequence are a causal decode
+    N, d = 37, 8
+    q, k, v = rand((2, 2, N, d), 54), rand((2, 1, N, d), 55), rand((2, 1, N, d), 56)
+    for causal in (True, False):
+        o, lse = oracle.decode_fwd64(q, k, v, causal, scale)
+        o2, lse2 = A.attention_fwd64(q, k, v, causal, scale)
+        np.testing.assert_allclose(o, o2, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse, lse2, rtol=1e-12)
+    o, lse = oracle.decode_fwd64(q[:, :, -5:], k, v, True, scale)
+    o2, lse2 = A.attention_fwd64(q, k, v, True, scale)
+    np.testing.assert_allclose(o, o2[:, :, -5:], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, lse2[:, :, -5:], rtol=1e-12)
+    # a single causal query is the last position: it sees every key
+    oc, lc = oracle.decode_fwd64(q[:, :, :1], k, v, True, scale)
+    on, ln = oracle.decode_fwd64(q[:, :, :1], k, v, False, scale)
+    np.testing.assert_allclose(oc, on, rtol=1e-12)
+    np.testing.assert_allclose(lc, ln, rtol=1e-12)
+
+
 def test_synth_e4m3_rounding_matches_torch():
     import torch
     x = np.random.default_rng(6).standard_normal(20000).astype(np.float32)
