@@ -411,6 +411,128 @@ def run_ours(args, w, world, rank, local):
 
 
 # ---------------------------------------------------------------------------
+# decode workload (one new query per head against a long K/V cache)
+# ---------------------------------------------------------------------------
+
+DECODE_METRIC = "attention decode: K/V cache bytes read per second on 1 B200 (% of measured HBM bandwidth)"
+
+
+def oracle_decode_head(w, q, k, v, b, h):
+    import numpy as np
+    import oracle
+    kvh = h // w.group
+    t0 = time.perf_counter()
+    oracle.decode_fwd64(q[b:b + 1, h:h + 1].astype(np.float64), k[b:b + 1, kvh:kvh + 1], v[b:b + 1, kvh:kvh + 1],
+                        w.causal, w.scale)
+    return time.perf_counter() - t0
+
+
+def run_decode(args, w, world, rank, local):
+    import torch
+
+    import exact_io_aware_44_b200 as fa
+    import synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    q, k, v = synth.decode_inputs(w)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        heads, tot = 0, 0.0
+        while heads < w.B * w.Hq and (heads == 0 or tot < args.cpu_budget):
+            b, h = divmod(heads, w.Hq)
+            tot += oracle_decode_head(w, q, k, v, b, h)
+            heads += 1
+        per_head_bytes = 2 * w.Nk * w.d * 2
+        cpu = {"value": round(heads * per_head_bytes / tot / 1e9, 3), "unit": "GB/s", "cores": blas_threads(),
+               "kind": "oracle", "sample": f"{heads} of {w.B * w.Hq} query heads, float64 NumPy (each head reads "
+                                           f"its kv head's cache)", "seconds": round(tot, 3)}
+    host_q = torch.from_numpy(q).to(torch.bfloat16).pin_memory()
+    dq = host_q.to(dev)
+    dk = torch.from_numpy(k).to(torch.bfloat16).to(dev)
+    dv = torch.from_numpy(v).to(torch.bfloat16).to(dev)
+    del k, v
+    o = torch.empty_like(dq)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d), dtype=torch.uint8, device=dev)
+    P = lambda t: t.data_ptr()
+
+    def step():
+        rc = fa.decode_raw(P(dq), P(dk), P(dv), P(o), P(lse), P(ws), w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
+                           w.scale, 0, sp)
+        if rc:
+            raise fa.FAError(rc, "fa_decode")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.get_status():
+        raise fa.FAError(fa.get_status(), "warm-up")
+    K = args.steps
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    if fa.get_status():
+        raise fa.FAError(fa.get_status(), "timed region")
+    ms = reduce_max(e0.elapsed_time(e1) / K)
+    kv_bytes = w.kv_bytes()
+    algo_bytes = kv_bytes + 2 * dq.numel() * 2 + lse.numel() * 4  # K, V read; q read, o written; lse
+    gbs = algo_bytes / (ms / 1e3) / 1e9
+    value = world * gbs
+    e2e = None
+    if not args.no_e2e:  # the cache stays on the device; each step brings its queries and returns o, lse
+        out_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        out_l = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        Ke = max(1, min(K, args.e2e_steps))
+        barrier()
+        torch.cuda.synchronize()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(Ke):
+            dq.copy_(host_q, non_blocking=True)
+            step()
+            out_o.copy_(o, non_blocking=True)
+            out_l.copy_(lse, non_blocking=True)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = reduce_max(a0.elapsed_time(a1) / Ke)
+        e2e = {"value": round(world * algo_bytes / (e_ms / 1e3) / 1e9, 1), "unit": "GB/s",
+               "h2d_bytes_per_step": host_q.numel() * 2, "d2h_bytes_per_step": out_o.numel() * 2 + out_l.numel() * 4,
+               "ms_per_step": round(e_ms, 4), "steps": Ke}
+    return {
+        "metric": DECODE_METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}: decode B={w.B} Hq={w.Hq} Hkv={w.Hkv} Nq={w.Nq} Nk={w.Nk} d={w.d} "
+                               f"{'causal' if w.causal else 'non-causal'} bf16",
+                   "l2": f"inputs larger than L2 (K and V caches {kv_bytes / 1e9:.2f} GB; L2 is 126 MB)",
+                   "parallelism": f"replicas x{world}"},
+        "tflops": round(w.flops() / (ms / 1e3) / 1e12, 2),
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(gbs / hbm, 4), "traffic": None, "kernel": "decode_split+merge",
+                     "peak_source": f"{peak_src} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clocks.summary(),
+    }
+
+
+# ---------------------------------------------------------------------------
 # reference arm: the float64 oracle as it stands, on the host cores
 # ---------------------------------------------------------------------------
 
@@ -438,6 +560,29 @@ def run_reference(args, w):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_reference_decode(args, w):
+    import synth
+    q, k, v = synth.decode_inputs(w)
+    times = []
+    for i in range(args.warmup + args.steps):
+        b, h = divmod(i % (w.B * w.Hq), w.Hq)
+        dt = oracle_decode_head(w, q, k, v, b, h)
+        if i >= args.warmup:
+            times.append(dt)
+    per_head_bytes = 2 * w.Nk * w.d * 2
+    ms = 1e3 * statistics.mean(times)
+    value = per_head_bytes / (ms / 1e3) / 1e9
+    sample = f"one query head per step: its decode against N_k={w.Nk} cached keys (d={w.d}) in float64"
+    return {"metric": DECODE_METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w.name}: decode B={w.B} Hq={w.Hq} Hkv={w.Hkv} Nq={w.Nq} Nk={w.Nk} d={w.d} "
+                                   f"(sampled per step)"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "kind": "oracle", "cores": blas_threads(),
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -445,7 +590,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c3",
-                    help="c2, c3, c5 (bf16 fwd+bwd), c4 (bf16 fwd), f3, f4 (E4M3 fwd)")
+                    help="c2, c3, c5 (bf16 fwd+bwd), c4 (bf16 fwd), f3, f4 (E4M3 fwd), dec (decode)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
@@ -455,8 +600,30 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
 
     import synth
-    w = synth.WORKLOADS[args.workload]
     world, rank, local = dist_env()
+    if args.workload in synth.DECODE_WORKLOADS:
+        w = synth.DECODE_WORKLOADS[args.workload]
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps(run_reference_decode(args, w)), flush=True)
+            return 0
+        import torch
+        torch.cuda.set_device(local)
+        if world > 1:
+            import torch.distributed as dist
+            from datetime import timedelta
+            dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+        try:
+            res = run_decode(args, w, world, rank, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                if dist.is_initialized():
+                    dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return 0
+    w = synth.WORKLOADS[args.workload]
 
     if args.impl == "reference":
         if rank == 0:

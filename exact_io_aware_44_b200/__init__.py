@@ -18,7 +18,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["fwd", "fwd_fp8", "bwd", "fwd_raw", "fwd_fp8_raw", "bwd_raw", "bwd_phases_raw", "workspace_bytes", "get_status", "set_wait_budget_ns",
+__all__ = ["fwd", "fwd_fp8", "decode", "decode_raw", "decode_workspace_bytes", "bwd", "fwd_raw", "fwd_fp8_raw", "bwd_raw", "bwd_phases_raw", "workspace_bytes", "get_status", "set_wait_budget_ns",
            "selftest_wait_timeout", "FAError", "LIB_PATH", "lib", "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
@@ -35,6 +35,8 @@ SIGNATURES = {
     "fa_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_fwd_fp8": (_I, [_P, _P, _P, _F, _F, _F, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "fa_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
+    "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_preprocess": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "fa_bwd_main": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
@@ -164,6 +166,43 @@ def fwd_fp8(q, k, v, descale_q: float, descale_k: float, descale_v: float, causa
     _require(lse, "lse", torch.float32, q.device)
     _check(lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), float(descale_q), float(descale_k), float(descale_v), _ptr(out),
                           _ptr(lse), B, Hq, Hkv, N, d, int(bool(causal)), scale, _stream_ptr(stream)), "fa_fwd_fp8")
+    return out, lse
+
+
+def decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits=0) -> int:
+    return int(lib.fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, int(num_splits)))
+
+
+def decode_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, ws_ptr, B, Hq, Hkv, Nq, Nk, d, causal, scale, num_splits,
+               stream_ptr):
+    """fa_decode on raw device pointers (ints); returns the status code."""
+    return lib.fa_decode(_P(q_ptr), _P(k_ptr), _P(v_ptr), _P(o_ptr), _P(lse_ptr), _P(ws_ptr), B, Hq, Hkv, Nq, Nk,
+                         d, int(bool(causal)), float(scale), int(num_splits), _P(stream_ptr))
+
+
+def decode(q, k, v, causal: bool = True, scale: float | None = None, num_splits: int = 0, out=None, lse=None,
+           workspace=None, stream=None):
+    """Attention of q [B, Hq, Nq, d] (the last Nq positions) against a key/value
+    cache k, v [B, Hkv, Nk, d], all bf16, split along the keys. Returns (o, lse)."""
+    import torch
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, N, d]")
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, dk) != (B, d) or v.shape != k.shape:
+        raise ValueError("k, v must be [B, Hkv, Nk, d] with q's B and d")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n, torch.bfloat16, q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits)
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    _check(lib.fa_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(workspace), B, Hq, Hkv, Nq, Nk, d,
+                         int(bool(causal)), scale, int(num_splits), _stream_ptr(stream)), "fa_decode")
     return out, lse
 
 

@@ -6,6 +6,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -227,6 +228,95 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   if (launch_fwd_f32(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+}  // extern "C"
+
+namespace fa {
+namespace {
+
+// Key splits for decode: enough (batch, kv head, split) CTAs for two per SM of a
+// 148-SM part, at most one split per 128-key chunk, and no empty split. A fixed
+// rule (not the current device's SM count) so that the workspace size can be
+// computed without a device.
+constexpr int kDecodeTargetCtas = 296;
+constexpr int kDecodeMaxSplits = 256;
+
+struct DecodeSplit {
+  int n_splits, chunks_per_split;
+};
+
+DecodeSplit decode_split(int B, int Hkv, int Nk, int num_splits) {
+  const int n_chunks = (Nk + kTileN - 1) / kTileN;
+  const long long base = (long long)B * Hkv;
+  long long want = num_splits > 0 ? num_splits : (kDecodeTargetCtas + base - 1) / base;
+  want = std::max(1LL, std::min<long long>({want, (long long)n_chunks, (long long)kDecodeMaxSplits}));
+  const int cps = (int)((n_chunks + want - 1) / want);
+  return {(n_chunks + cps - 1) / cps, cps};
+}
+
+int check_decode(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale) {
+  bool empty;
+  int rc = check_sizes(B, Hq, Hkv, Nq, d, scale, &empty);
+  if (rc != FA_OK) return rc;
+  if (Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  if (causal && Nq > Nk) return FA_ERR_INVALID_ARG;
+  if (d != 128 || (Hq / Hkv) * Nq > 16) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * Hkv * (long long)Nk >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+size_t decode_workspace(int B, int Hq, int Nq, int d, const DecodeSplit& sp) {
+  const size_t rows = (size_t)B * Hq * Nq;
+  const size_t opart = ((size_t)sp.n_splits * rows * d * sizeof(float) + 255) & ~size_t(255);
+  return opart + (size_t)sp.n_splits * rows * sizeof(float);
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {
+  if (check_decode(B, Hq, Hkv, Nq, Nk, d, 0, 1.f) != FA_OK) return 0;
+  return decode_workspace(B, Hq, Nq, d, decode_split(B, Hkv, Nk, num_splits));
+}
+
+int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace, int B, int Hq,
+              int Hkv, int Nq, int Nk, int d, int causal, float scale, int num_splits, void* stream) {
+  int rc = check_decode(B, Hq, Hkv, Nq, Nk, d, causal, scale);
+  if (rc != FA_OK) return rc;
+  if (!q || !k || !v || !o || !lse || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_ALIGNMENT;
+  DeviceInfo* di;
+  if ((rc = current_device(&di)) != FA_OK) return rc;
+  const DecodeSplit sp = decode_split(B, Hkv, Nk, num_splits);
+  const long long rows = (long long)B * Hq * Nq;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_map(&tq, q, d, (int)rows, 1, 16)) != FA_OK) return rc;
+  if ((rc = make_map(&tk, k, d, Nk, B * Hkv)) != FA_OK) return rc;
+  if ((rc = make_map(&tv, v, d, Nk, B * Hkv)) != FA_OK) return rc;
+  DecodeParams p;
+  p.o = o;
+  p.lse = lse;
+  p.o_part = static_cast<float*>(workspace);
+  const size_t opart = ((size_t)sp.n_splits * rows * d * sizeof(float) + 255) & ~size_t(255);
+  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + opart);
+  p.status = di->status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.causal = causal ? 1 : 0;
+  p.n_splits = sp.n_splits;
+  p.chunks_per_split = sp.chunks_per_split;
+  p.rows_total = rows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_budget_ns = g_wait_budget_ns.load();
+  if (launch_decode(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
 }
 

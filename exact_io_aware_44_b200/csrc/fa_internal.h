@@ -46,12 +46,29 @@ struct BwdParams {
   uint64_t wait_budget_ns;
 };
 
+struct DecodeParams {
+  void* o;            // bf16 [B, Hq, Nq, d]
+  float* lse;         // [B, Hq, Nq]
+  float* o_part;      // workspace: per split, normalised partial O [n_splits, B * Hq * Nq, d]
+  float* lse_part;    // workspace: per split, partial LSE (natural log) [n_splits, B * Hq * Nq]
+  int* status;
+  int B, Hq, Hkv, Nq, Nk;
+  int causal;
+  int n_splits, chunks_per_split;  // key splits and 128-key chunks per split
+  long long rows_total;            // B * Hq * Nq
+  float scale_log2;
+  uint64_t wait_budget_ns;
+};
+
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int d, cudaStream_t s);
 cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, cudaStream_t s);
 cudaError_t launch_fwd_f32(const FwdF32Params& p, cudaStream_t s);
+// Decode: the split kernel, then the merge of the splits.
+cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                          cudaStream_t s);
 // Query rows per tile of the main backward kernel for head dim d (its TMA box height).
 int bwd_query_rows(int d);
 // Backward phases: D and zeroed dQ accumulator; main kernel; dQ conversion.

@@ -99,6 +99,43 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, flo
                void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * fa_decode_workspace_bytes -- device scratch that fa_decode needs.
+ *
+ * Per key split, a float32 partial output [B*Hq*Nq, d] and a float32 partial
+ * LSE [B*Hq*Nq]. num_splits <= 0 means the split count fa_decode chooses itself
+ * (a fixed rule of the sizes, so no device is needed here). Returns 0 for sizes
+ * fa_decode rejects.
+ */
+size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits);
+
+/*
+ * fa_decode -- attention of Nq new queries against a cache of Nk keys and values,
+ * split along the keys (decode).
+ *
+ * In serving the kernel runs against a KV cache, and the decode step is bound by
+ * reading that cache ("FlashAttention Kernel & Online Softmax" card: KV cache and
+ * the decode bandwidth bottleneck). The queries are the last Nq positions of the
+ * sequence: query i is at position Nk - Nq + i and, when causal != 0, sees keys
+ * j <= Nk - Nq + i (Nq = Nk gives fa_fwd's square causal mask). Each key split
+ * computes a partial softmax over its keys; the partials are combined with the
+ * online-softmax merge (running max, rescaled denominators: the update of the
+ * card's first paragraph), LSE = log sum_s e^(LSE_s), O = sum_s e^(LSE_s - LSE) O_s.
+ *   q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] bf16   inputs (read only)
+ *   o [B,Hq,Nq,d] bf16, lse [B,Hq,Nq] float32   outputs, as in fa_fwd
+ *   workspace   at least fa_decode_workspace_bytes(..., num_splits) bytes of
+ *               device memory, 256-byte aligned, contents on entry irrelevant
+ *   num_splits  key splits (<= 0: chosen from the sizes; capped by the number of
+ *               128-key chunks)
+ *   d must be 128 and (Hq / Hkv) * Nq at most 16 (one CTA serves a whole GQA
+ *   group's query rows), else FA_ERR_UNSUPPORTED; causal with Nq > Nk is
+ *   FA_ERR_INVALID_ARG. Arithmetic: bf16 operands, fp32 accumulation; P is
+ *   rounded to bf16 before the P V product; the partials stay fp32.
+ */
+int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
+              int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale, int num_splits,
+              void* stream);
+
+/*
  * fa_fwd_f32 -- float32 forward pass (CUDA cores, fp32 throughout).
  *
  * The same computation as fa_fwd, on float32 q, k, v and o. Tiles of queries

@@ -24,6 +24,7 @@ Workloads (shapes from the pages' long-context regime; all synthetic, no dataset
   c5  bf16 fwd+bwd GQA, B=1 Hq=32 Hkv=8 N=32768 d=128, causal
   f3  E4M3 fwd,  B=2 H=32 N=8192 d=128, causal, std 1/sqrt(2) (c3's shape)
   f4  E4M3 fwd,  B=1 H=16 N=65536 d=128, causal (c4's shape)
+  dec decode,    B=16 Hq=32 Hkv=8, Nq=1 new query against Nk=32768 cached keys, d=128
 """
 from __future__ import annotations
 
@@ -185,6 +186,62 @@ def small(B, Hq, Hkv, N, d, causal, seed, dtype="bf16", std=1.0, backward=True,
     return Workload(f"t{B}x{Hq}x{Hkv}x{N}x{d}{'c' if causal else ''}", B, Hq, Hkv, N, d,
                     causal, dtype, backward, seed, std=std, spike_frac=spike_frac,
                     spike_mul=spike_mul)
+
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Nq new queries against a cache of Nk keys/values (bf16)."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    seed: int
+    std: float = 1.0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+    def flops(self) -> float:
+        return 4.0 * self.B * self.Hq * self.Nq * self.Nk * self.d
+
+    def kv_bytes(self) -> int:
+        return 2 * self.B * self.Hkv * self.Nk * self.d * 2
+
+
+DECODE_WORKLOADS = {
+    # one decode step of a GQA model (32 query heads, 8 kv heads) over a 32K-token cache
+    "dec": DecodeWorkload("dec", 16, 32, 8, 1, 32768, 128, True, 1010),
+}
+
+
+def decode_inputs(w: DecodeWorkload, workers: int | None = None):
+    """(q [B,Hq,Nq,d], k, v [B,Hkv,Nk,d]) float32, bf16-representable, one seeded
+    stream per (tensor, batch, head) as for the other workloads."""
+    def fill(args):
+        out, tid, b, h = args
+        x = _rng(w.seed, tid, b, h).standard_normal(out.shape[2:], dtype=np.float32)
+        if w.std != 1.0:
+            x *= np.float32(w.std)
+        out[b, h] = round_to_bf16(x)
+
+    q = np.empty((w.B, w.Hq, w.Nq, w.d), dtype=np.float32)
+    k = np.empty((w.B, w.Hkv, w.Nk, w.d), dtype=np.float32)
+    v = np.empty_like(k)
+    jobs = [(q, TID_Q, b, h) for b in range(w.B) for h in range(w.Hq)]
+    jobs += [(t, tid, b, h) for t, tid in ((k, TID_K), (v, TID_V)) for b in range(w.B) for h in range(w.Hkv)]
+    workers = workers or min(len(jobs), os.cpu_count() or 1)
+    with _cf.ThreadPoolExecutor(workers) as ex:
+        list(ex.map(fill, jobs))
+    return q, k, v
 
 
 def sample_rows(w: Workload, b: int, h: int, count: int | None = None) -> np.ndarray:

@@ -81,6 +81,39 @@ def test_fp8_forward_rejects_bad_arguments_on_host():
     assert _fwd8(N=0, ptr=0) == 0
 
 
+def _dec(B=1, Hq=8, Hkv=1, Nq=1, Nk=1000, d=128, causal=1, scale=0.088, splits=0, ptr=0x1000, ws=0x1000):
+    return fa.decode_raw(ptr, ptr, ptr, ptr, ptr, ws, B, Hq, Hkv, Nq, Nk, d, causal, scale, splits, 0)
+
+
+def test_decode_rejects_bad_arguments_on_host():
+    assert _dec(d=64) == -2                        # d = 128 only
+    assert _dec(Hq=32, Hkv=1) == -2                # 32 query rows per group > 16
+    assert _dec(Hq=8, Nq=3) == -2                  # 24 rows > 16
+    assert _dec(Nq=5, Nk=4) == -1                  # causal needs Nq <= Nk
+    assert _dec(Nk=0) == -1
+    assert _dec(Hq=6, Hkv=4) == -1
+    assert _dec(scale=float("nan")) == -1
+    assert _dec(ws=0x1010) == -3                   # workspace 256-byte aligned
+    assert _dec(ptr=0x1008) == -3
+    assert _dec(ws=0) == -1
+
+
+def test_decode_workspace_and_split_rule():
+    """Per split: fp32 partial O (256-byte padded) and fp32 partial LSE per query row."""
+    B, Hq, Hkv, Nq, d = 4, 32, 8, 1, 128
+    for Nk, splits in ((128, 1), (4096, 4), (4096, 7), (100000, 0)):
+        ws = fa.decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, splits)
+        n_chunks = -(-Nk // 128)
+        want = splits if splits > 0 else -(-296 // (B * Hkv))
+        want = max(1, min(want, n_chunks, 256))
+        cps = -(-n_chunks // want)
+        ns = -(-n_chunks // cps)
+        rows = B * Hq * Nq
+        opart = (ns * rows * d * 4 + 255) // 256 * 256
+        assert ws == opart + ns * rows * 4, (Nk, splits, ws)
+    assert fa.decode_workspace_bytes(1, 8, 1, 1, 1000, 64, 0) == 0
+
+
 def test_bwd_rejects_bad_arguments_on_host():
     p = 0x1000
     r = fa.bwd_raw(p, p, p, p, p, p, p, p, p, p + 16, 1, 2, 1, 128, 64, 1, 0.125, 0)
