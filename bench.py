@@ -226,7 +226,9 @@ def cpu_baseline(w, budget_s: float = 15.0):
         total_f += f
         heads += 1
     what = "forward + backward" if w.backward else "forward"
+    full_f = (w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0))
     return {"value": total_f / total_t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "full_problem_seconds_extrapolated": round(full_f / (total_f / total_t), 1),
             "sample": f"{heads} of {w.B * w.Hq} (batch, head) pairs, full {what} each, float64 NumPy",
             "seconds": round(total_t, 3)}
 
@@ -325,10 +327,9 @@ def run_ours(args, w, world, rank, local):
     ms_total = t_start.elapsed_time(t_end)
     ms_step = reduce_max(ms_total / K)
     # events: 0 fwd start, 1 bwd pre start (= fwd end), 2 main start, 3 convert start, 4 bwd end
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    pre_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    conv_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
+    per_kernel = {name: [e[i].elapsed_time(e[i + 1]) for e in evs]
+                  for i, name in enumerate(("fwd", "bwd_preprocess", "bwd_main", "bwd_convert"))}
+    fwd_ms, pre_ms, main_ms, conv_ms = (statistics.mean(per_kernel[n]) for n in per_kernel)
     f_fwd, f_bwd = w.fwd_flops(), (w.bwd_flops() if w.backward else 0.0)
     value = job_throughput(f_fwd + f_bwd, world, ms_step / 1e3)
 
@@ -401,6 +402,19 @@ def run_ours(args, w, world, rank, local):
         "fwd_tflops": round(kernels["fwd"]["tflops"], 1),
         "bwd_tflops": round(f_bwd / (pre_ms + main_ms + conv_ms) / 1e9, 1) if w.backward else None,
         "kernels_ms": {k: round(v["ms"], 4) for k, v in kernels.items()},
+        "kernels_ms_median_min": {k: [round(statistics.median(v), 4), round(min(v), 4)]
+                                  for k, v in per_kernel.items() if (w.backward or k == "fwd")},
+        # The pages' traffic argument: standard attention writes the N x N scores and
+        # reads them back (fp16 S and P, each written and read once: 8 B*Hq*N^2 bytes);
+        # this path moves only the O(N) tensors (algorithmic bytes; ncu-measured DRAM
+        # bytes of the dominant kernel in `roofline.traffic`).
+        "traffic_model": {"standard_attention_bytes": 8 * B * Hq * N * N,
+                          # Q, K, V read (input dtype), O written (bf16), LSE written (fp32)
+                          "fwd_algorithmic_bytes": (B * Hq + 2 * B * Hkv) * N * d * (1 if fp8 else 2)
+                          + B * Hq * N * d * 2 + B * Hq * N * 4,
+                          "bwd_workspace_bytes": fa.workspace_bytes(B, Hq, Hkv, N, d) if w.backward else 0,
+                          "note": "the workspace is linear in N (D and the fp32 dQ accumulator); "
+                                  "no N x N buffer exists"},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -111,7 +111,7 @@ def sampled_bwd_check(w, device):
     return worst
 
 
-@pytest.mark.parametrize("name", ["c3", "c5"])
+@pytest.mark.parametrize("name", ["c3", "c3n", "c5"])
 def test_bf16_bwd_full_size_sampled(cuda_device, name):
     sampled_bwd_check(synth.WORKLOADS[name], cuda_device)
 

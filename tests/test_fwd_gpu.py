@@ -172,7 +172,7 @@ def sampled_fwd_check(w, device):
     return worst
 
 
-@pytest.mark.parametrize("name", ["c3", "c4", "c5"])
+@pytest.mark.parametrize("name", ["c3", "c3n", "c4", "c5"])
 def test_bf16_fwd_full_size_sampled(cuda_device, name):
     sampled_fwd_check(synth.WORKLOADS[name], cuda_device)
 
