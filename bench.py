@@ -262,10 +262,21 @@ def run_ours(args, w, world, rank, local):
     host = {}
     tids = (("q", synth.TID_Q), ("k", synth.TID_K), ("v", synth.TID_V)) + ((("do", synth.TID_DO),) if w.backward else ())
     in_dtype = torch.float8_e4m3fn if fp8 else torch.bfloat16
-    for name, tid in tids:
-        host[name] = torch.from_numpy(synth.tensor(w, tid)).to(in_dtype).pin_memory()
-    d_in = {n: t.to(dev) for n, t in host.items()}
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    share = 1.0
+    if args.shard == "heads":
+        # strong scaling: this rank computes its slice of the flattened head axis
+        q0, q1, k0, k1 = fa.head_shard(B, Hq, Hkv, rank, world)
+        share = (k1 - k0) / (B * Hkv)
+    for name, tid in tids:
+        x = synth.tensor(w, tid)
+        if args.shard == "heads":
+            lo, hi = (q0, q1) if name in ("q", "do") else (k0, k1)
+            x = x.reshape(B * x.shape[1], N, d)[lo:hi][None]
+        host[name] = torch.from_numpy(np.ascontiguousarray(x)).to(in_dtype).pin_memory()
+    d_in = {n: t.to(dev) for n, t in host.items()}
+    if args.shard == "heads":
+        B, Hq, Hkv = 1, q1 - q0, k1 - k0
     o = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
     if w.backward:
@@ -330,8 +341,11 @@ def run_ours(args, w, world, rank, local):
     per_kernel = {name: [e[i].elapsed_time(e[i + 1]) for e in evs]
                   for i, name in enumerate(("fwd", "bwd_preprocess", "bwd_main", "bwd_convert"))}
     fwd_ms, pre_ms, main_ms, conv_ms = (statistics.mean(per_kernel[n]) for n in per_kernel)
-    f_fwd, f_bwd = w.fwd_flops(), (w.bwd_flops() if w.backward else 0.0)
-    value = job_throughput(f_fwd + f_bwd, world, ms_step / 1e3)
+    f_fwd, f_bwd = w.fwd_flops() * share, (w.bwd_flops() * share if w.backward else 0.0)
+    if args.shard == "heads":  # the ranks' shares add up to one workload
+        value = (w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)) / (ms_step / 1e3) / 1e12
+    else:
+        value = job_throughput(f_fwd + f_bwd, world, ms_step / 1e3)
 
     kernels = {
         "fwd": {"ms": fwd_ms, "tflops": f_fwd / fwd_ms / 1e9},
@@ -378,7 +392,9 @@ def run_ours(args, w, world, rank, local):
         torch.cuda.synchronize()
         barrier()
         e_ms = reduce_max(e0.elapsed_time(e1) / Ke)
-        e2e = {"value": round(job_throughput(f_fwd + f_bwd, world, e_ms / 1e3), 2), "unit": UNIT,
+        e2e_value = ((w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)) / (e_ms / 1e3) / 1e12
+                     if args.shard == "heads" else job_throughput(f_fwd + f_bwd, world, e_ms / 1e3))
+        e2e = {"value": round(e2e_value, 2), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 3),
                "steps": Ke}
         st = fa.get_status()
@@ -388,7 +404,8 @@ def run_ours(args, w, world, rank, local):
     clk = clocks.summary()
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "strong" if args.shard == "heads" else "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": f"{w.name}: B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} "
                                f"{'causal' if w.causal else 'non-causal'} {w.dtype} "
@@ -397,7 +414,7 @@ def run_ours(args, w, world, rank, local):
                    "l2": "inputs larger than L2 ("
                          + ("Q, K, V, O, dO are" if w.backward else "Q, K, V are")
                          + f" {B * Hq * N * d * (1 if fp8 else 2) / 1e6:.0f} MB each; L2 is 126 MB)",
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": f"head shards x{world}" if args.shard == "heads" else f"replicas x{world}"},
         "pct_of_peak": round(100 * value / world / peak, 2),
         "fwd_tflops": round(kernels["fwd"]["tflops"], 1),
         "bwd_tflops": round(f_bwd / (pre_ms + main_ms + conv_ms) / 1e9, 1) if w.backward else None,
@@ -605,6 +622,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c3",
                     help="c2, c3, c5 (bf16 fwd+bwd), c4 (bf16 fwd), f3, f4 (E4M3 fwd), dec (decode)")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N>1: every rank runs the whole workload (weak scaling) or its slice of the heads (strong)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")

@@ -18,7 +18,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["fwd", "fwd_fp8", "decode", "decode_raw", "decode_workspace_bytes", "bwd", "fwd_raw", "fwd_fp8_raw", "bwd_raw", "bwd_phases_raw", "workspace_bytes", "get_status", "set_wait_budget_ns",
+__all__ = ["head_shard", "fwd", "fwd_fp8", "decode", "decode_raw", "decode_workspace_bytes", "bwd", "fwd_raw", "fwd_fp8_raw", "bwd_raw", "bwd_phases_raw", "workspace_bytes", "get_status", "set_wait_budget_ns",
            "selftest_wait_timeout", "FAError", "LIB_PATH", "lib", "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
@@ -167,6 +167,27 @@ def fwd_fp8(q, k, v, descale_q: float, descale_k: float, descale_v: float, causa
     _check(lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), float(descale_q), float(descale_k), float(descale_v), _ptr(out),
                           _ptr(lse), B, Hq, Hkv, N, d, int(bool(causal)), scale, _stream_ptr(stream)), "fa_fwd_fp8")
     return out, lse
+
+
+def head_shard(B: int, Hq: int, Hkv: int, rank: int, world: int):
+    """The query and key/value heads one rank computes when a problem is split
+    across `world` GPUs by heads (no exchange between ranks: every (batch, kv head)
+    group is independent in the forward and the backward).
+
+    Heads are counted on the flattened [B * H] axis of the [B, H, N, d] layout, so
+    a rank's share is one contiguous slice: query heads [q0, q1) and kv heads
+    [k0, k1), cut at GQA group boundaries, with group counts differing by at most
+    one between ranks. The slice is a valid problem of its own with B = 1,
+    Hq = q1 - q0, Hkv = k1 - k0 (query head i of the slice reads kv head
+    i // (Hq / Hkv) of its slice). Returns (q0, q1, k0, k1); an empty slice when
+    world exceeds the number of groups."""
+    if world < 1 or not 0 <= rank < world or Hkv < 1 or Hq % Hkv:
+        raise ValueError("invalid shard request")
+    groups, g = B * Hkv, Hq // Hkv
+    base, extra = divmod(groups, world)
+    k0 = rank * base + min(rank, extra)
+    k1 = k0 + base + (1 if rank < extra else 0)
+    return k0 * g, k1 * g, k0, k1
 
 
 def decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits=0) -> int:
