@@ -48,6 +48,8 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 NCU_TRAFFIC = {
     # profiles/bwd_main_d128_B2H32N8192_causal.md
     ("bwd_main", "c3"): {"bytes_per_launch": 809986560 + 491049984, "csrc_sha": "7497d3bd4abc43c9"},
+    # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md
+    ("decode_split", "dec"): {"bytes_per_launch": 2147724544 + 4109568, "csrc_sha": "812f00ecc35581b6"},
 }
 
 
@@ -58,6 +60,7 @@ KERNEL_SOURCES = {
     "bwd_main": ("fa_bwd_sm100.cu", [("__device__ __forceinline__ void red_add_v4", "// ----"),
                                      ("struct Bwd128Cfg {", "int sm_count() {")]),
     "fwd": ("fa_fwd_sm100.cu", [("", None)]),
+    "decode_split": ("fa_decode_sm100.cu", [("", None)]),
 }
 
 
@@ -519,6 +522,8 @@ def run_decode(args, w, world, rank, local):
         raise fa.FAError(fa.get_status(), "timed region")
     ms = reduce_max(e0.elapsed_time(e1) / K)
     kv_bytes = w.kv_bytes()
+    rec = NCU_TRAFFIC.get(("decode_split", w.name))
+    traffic = rec["bytes_per_launch"] if rec and rec.get("csrc_sha") == kernel_source_hash("decode_split") else None
     algo_bytes = kv_bytes + 2 * dq.numel() * 2 + lse.numel() * 4  # K, V read; q read, o written; lse
     gbs = algo_bytes / (ms / 1e3) / 1e9
     value = world * gbs
@@ -554,7 +559,7 @@ def run_decode(args, w, world, rank, local):
                    "parallelism": f"replicas x{world}"},
         "tflops": round(w.flops() / (ms / 1e3) / 1e12, 2),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(gbs / hbm, 4), "traffic": None, "kernel": "decode_split+merge",
+                     "frac": round(gbs / hbm, 4), "traffic": traffic, "kernel": "decode_split+merge",
                      "peak_source": f"{peak_src} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
         "cpu_baseline": cpu,
         "e2e": e2e,
