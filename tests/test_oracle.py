@@ -297,13 +297,14 @@ def test_head_probs_are_the_softmax_of_brute_force_scores():
         np.testing.assert_allclose(p @ v, np.array(o_ref)[sel], rtol=1e-10, atol=1e-12)
 
 
-def test_decode_oracle_pins():
+def pin_decode(dec):
+    """Pins for a decode implementation dec(q, k, v, causal, scale) -> (O, LSE)."""
     scale = 0.35
     # brute force on tiny shapes, GQA, causal and not
     for causal in (True, False):
         for (Nq, Nk) in ((1, 1), (1, 5), (3, 7), (4, 4)):
             q, k, v = rand((1, 4, Nq, 3), 51), rand((1, 2, Nk, 3), 52), rand((1, 2, Nk, 3), 53)
-            o, lse = oracle.decode_fwd64(q, k, v, causal, scale)
+            o, lse = dec(q, k, v, causal, scale)
             for h in range(4):
                 ob, lb = oracle.decode_naive_loops(q[0, h].tolist(), k[0, h // 2].tolist(), v[0, h // 2].tolist(),
                                                     causal, scale)
@@ -313,19 +314,59 @@ def test_decode_oracle_pins():
     N, d = 37, 8
     q, k, v = rand((2, 2, N, d), 54), rand((2, 1, N, d), 55), rand((2, 1, N, d), 56)
     for causal in (True, False):
-        o, lse = oracle.decode_fwd64(q, k, v, causal, scale)
+        o, lse = dec(q, k, v, causal, scale)
         o2, lse2 = A.attention_fwd64(q, k, v, causal, scale)
         np.testing.assert_allclose(o, o2, rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(lse, lse2, rtol=1e-12)
-    o, lse = oracle.decode_fwd64(q[:, :, -5:], k, v, True, scale)
+    o, lse = dec(q[:, :, -5:], k, v, True, scale)
     o2, lse2 = A.attention_fwd64(q, k, v, True, scale)
     np.testing.assert_allclose(o, o2[:, :, -5:], rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(lse, lse2[:, :, -5:], rtol=1e-12)
     # a single causal query is the last position: it sees every key
-    oc, lc = oracle.decode_fwd64(q[:, :, :1], k, v, True, scale)
-    on, ln = oracle.decode_fwd64(q[:, :, :1], k, v, False, scale)
+    oc, lc = dec(q[:, :, :1], k, v, True, scale)
+    on, ln = dec(q[:, :, :1], k, v, False, scale)
     np.testing.assert_allclose(oc, on, rtol=1e-12)
     np.testing.assert_allclose(lc, ln, rtol=1e-12)
+
+
+def test_decode_oracle_pins():
+    pin_decode(oracle.decode_fwd64)
+
+
+def _mut_decode_top_left(q, k, v, causal, scale=None):
+    """Queries aligned to the start of the cache (query i sees keys j <= i)."""
+    q, k, v = (np.asarray(x, float) for x in (q, k, v))
+    B, Hq, Nq, d = q.shape
+    Nk = k.shape[2]
+    g = Hq // k.shape[1]
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            s = scale * q[b, h] @ k[b, h // g].T
+            if causal:
+                s = np.where(np.arange(Nk)[None, :] <= np.arange(Nq)[:, None], s, -np.inf)
+            m = s.max(1, keepdims=True)
+            l = np.exp(s - m).sum(1, keepdims=True)
+            o[b, h] = (np.exp(s - m) / l) @ v[b, h // g]
+            lse[b, h] = (m + np.log(l))[:, 0]
+    return o, lse
+
+
+def _mut_decode_gqa_modulo(q, k, v, causal, scale=None):
+    Hq, Hkv = np.asarray(q).shape[1], np.asarray(k).shape[1]
+    idx = [h % Hkv for h in range(Hq)]
+    return oracle.decode_fwd64(q, np.asarray(k)[:, idx], np.asarray(v)[:, idx], causal, scale)
+
+
+def _mut_decode_lse_log2(q, k, v, causal, scale=None):
+    o, lse = oracle.decode_fwd64(q, k, v, causal, scale)
+    return o, lse / math.log(2)
+
+
+@pytest.mark.parametrize("mutant", [_mut_decode_top_left, _mut_decode_gqa_modulo, _mut_decode_lse_log2])
+def test_planted_decode_mistakes_are_caught(mutant):
+    assert _fails(pin_decode, mutant), mutant.__name__
 
 
 def test_synth_e4m3_rounding_matches_torch():
