@@ -62,6 +62,10 @@ constexpr uint32_t kRescaleThresholdLog2 = 8;  // rescale only when m grows by >
 // Of every 8 key pairs, how many take 2^x by polynomial on the FMA pipe instead
 // of the SFU (0 = all on the SFU).
 constexpr int kPolyPairs = FA_FWD_POLY_PAIRS;
+#ifndef FA_FWD64_POLY_PAIRS
+#define FA_FWD64_POLY_PAIRS 2
+#endif
+constexpr int kPolyPairs64 = FA_FWD64_POLY_PAIRS;  // the same, for d = 64 (bf16)
 
 // D: head dim; FP8: E4M3 Q, K, V and P (kind::f8f6f4 MMAs), else bf16 (kind::f16).
 template <int D, bool FP8>
@@ -360,13 +364,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           f2_unpack(f2_fma(f2_pack(s[i], s[i + 1]), c2, nmc2), x0, x1);
           f2_unpack(f2_fma(f2_pack(s[i + 2], s[i + 3]), c2, nmc2), x2, x3);
           float e0, e1, e2, e3;
-          if (((i / 2) & 7) < kPolyPairs) {
+          if (((i / 2) & 7) < (D == 64 ? kPolyPairs64 : kPolyPairs)) {
             ex2_poly2(x0, x1, e0, e1);
           } else {
             e0 = ex2(x0);
             e1 = ex2(x1);
           }
-          if (((i / 2 + 1) & 7) < kPolyPairs) {
+          if (((i / 2 + 1) & 7) < (D == 64 ? kPolyPairs64 : kPolyPairs)) {
             ex2_poly2(x2, x3, e2, e3);
           } else {
             e2 = ex2(x2);
