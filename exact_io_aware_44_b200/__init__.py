@@ -115,7 +115,7 @@ def fwd_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, N, d, causal, scale
 
 
 def fwd(q, k, v, causal: bool = True, scale: float | None = None, out=None, lse=None, stream=None):
-    """Forward pass. bf16 inputs run on the tensor cores (d in {64, 128});
+    """Forward pass. bf16 inputs run on the tensor cores (d in {64, 128, 256});
     float32 inputs run the fp32 CUDA-core kernel. Returns (o, lse)."""
     import torch
     B, Hq, Hkv, N, d = _dims(q, k)

@@ -140,7 +140,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   bool empty;
   int rc = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
   if (rc != FA_OK) return rc;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   if (empty) return FA_OK;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
@@ -159,7 +159,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.Hkv = Hkv;
   p.N = N;
   p.causal = causal ? 1 : 0;
-  p.n_qblk = (N + 2 * kTileM - 1) / (2 * kTileM);
+  const int rows_per_cta = fwd_tiles_per_cta(d) * kTileM;
+  p.n_qblk = (N + rows_per_cta - 1) / rows_per_cta;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_scale = 1.f;
   p.wait_budget_ns = g_wait_budget_ns.load();

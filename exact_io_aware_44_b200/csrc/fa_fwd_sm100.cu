@@ -71,7 +71,10 @@ constexpr int kPolyPairs64 = FA_FWD64_POLY_PAIRS;  // the same, for d = 64 (bf16
 template <int D, bool FP8>
 struct FwdCfg {
   static constexpr int kElem = FP8 ? 1 : 2;                      // bytes per element
-  static constexpr int kStages = (FP8 || D == 64) ? 10 : 5;      // K/V ring: K_0, V_0, K_1, V_1, ...
+  // Query tiles per CTA: two, except d = 256, whose O tile alone takes 256 TMEM columns.
+  static constexpr int kTiles = D == 256 ? 1 : 2;
+  // K/V ring: K_0, V_0, K_1, V_1, ... (d = 256: two 64 KB stages next to the 64 KB Q tile)
+  static constexpr int kStages = (FP8 || D == 64) ? 10 : (D == 256 ? 2 : 5);
   static constexpr int kTileBytes = kTileM * D * kElem;          // one Q, K or V tile
   static constexpr int kRegion = kTileM * 128;                   // one 128-byte-wide column block
   static constexpr int kRegions = D * kElem / 128;               // column blocks per tile
@@ -80,7 +83,7 @@ struct FwdCfg {
   static constexpr int kSSteps = D / kKStep;                     // MMAs per S tile
   static constexpr int kPvSteps = kTileN / kKStep;               // MMAs per P V (8 TMEM columns each)
   static constexpr int kOffQ = 0;
-  static constexpr int kOffKV = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffKV = kOffQ + kTiles * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
   // q_full, full[S], empty[S], s_ready[2], p_ready[2], o_done[2], mma_final
   static constexpr int kNumBars = 1 + 2 * kStages + 7;
@@ -121,13 +124,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int b = bh / p.Hq;
   const int h = bh % p.Hq;
   const int kv_head = b * p.Hkv + h / (p.Hq / p.Hkv);
-  const int q0 = qb * 2 * kTileM;
+  const int q0 = qb * C::kTiles * kTileM;
   const int n_kv_all = (p.N + kTileN - 1) / kTileN;
   int n_iter[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int qt = q0 / kTileM + t;  // index of this query tile
-    const bool active = q0 + t * kTileM < p.N;
+    const bool active = t < C::kTiles && q0 + t * kTileM < p.N;
     n_iter[t] = !active ? 0 : (p.causal ? qt + 1 : n_kv_all);
   }
   const int n_kv = max(n_iter[0], n_iter[1]);
@@ -473,8 +476,11 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int d, cudaStream_t s) {
+  if (d == 256) return launch_fwd_d<256, false>(tq, tk, tv, p, s);
   return d == 128 ? launch_fwd_d<128, false>(tq, tk, tv, p, s) : launch_fwd_d<64, false>(tq, tk, tv, p, s);
 }
+
+int fwd_tiles_per_cta(int d) { return d == 256 ? FwdCfg<256, false>::kTiles : 2; }
 
 cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, cudaStream_t s) {

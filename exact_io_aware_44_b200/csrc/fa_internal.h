@@ -63,6 +63,8 @@ struct DecodeParams {
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int d, cudaStream_t s);
+// Query tiles of 128 rows per forward CTA for head dim d (the grid's query blocks).
+int fwd_tiles_per_cta(int d);
 cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, cudaStream_t s);
 cudaError_t launch_fwd_f32(const FwdF32Params& p, cudaStream_t s);

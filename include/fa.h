@@ -69,8 +69,8 @@ typedef enum {
  *   q [B,Hq,N,d] bf16, k/v [B,Hkv,N,d] bf16   inputs (read only)
  *   o [B,Hq,N,d] bf16                          output, round-to-nearest-even
  *   lse [B,Hq,N] float32                       output
- *   d must be 64 or 128. Arithmetic: bf16 operands, fp32 accumulation; the
- *   probabilities P are rounded to bf16 before the P V product.
+ *   d must be 64, 128 or 256 (fa_bwd: 64 or 128). Arithmetic: bf16 operands, fp32
+ *   accumulation; the probabilities P are rounded to bf16 before the P V product.
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);

@@ -61,6 +61,23 @@ def test_bf16_fwd_small(cuda_device, shape, causal):
     check_full(w, cuda_device)
 
 
+D256_SHAPES = [
+    # B, Hq, Hkv, N (d = 256: one 128-row query tile per CTA)
+    (1, 1, 1, 1),
+    (1, 2, 1, 129),
+    (2, 2, 2, 300),
+    (1, 4, 2, 1000),
+]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("shape", D256_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_bf16_fwd_d256(cuda_device, shape, causal):
+    B, Hq, Hkv, N = shape
+    w = synth.small(B, Hq, Hkv, N, 256, causal, seed=900 + N)
+    check_full(w, cuda_device)
+
+
 def test_bf16_fwd_spiked_rows_force_rescales(cuda_device):
     """Query rows x20 make late key tiles raise the running max far above the
     lazy-rescale threshold."""
@@ -172,7 +189,7 @@ def sampled_fwd_check(w, device):
     return worst
 
 
-@pytest.mark.parametrize("name", ["c3", "c3n", "c4", "c5"])
+@pytest.mark.parametrize("name", ["c3", "c3n", "c4", "c5", "c6"])
 def test_bf16_fwd_full_size_sampled(cuda_device, name):
     sampled_fwd_check(synth.WORKLOADS[name], cuda_device)
 
