@@ -206,7 +206,7 @@ def oracle_head_step(w, b: int, h: int):
     import numpy as np
     import oracle
     import synth
-    ds = w.descale if w.dtype == "e4m3" else 1.0  # E4M3 slices hold codes; real value = code * descale
+    ds = w.descale if w.dtype in ("e4m3", "e5m2") else 1.0  # FP8 slices hold codes; real value = code * descale
     q = synth.head_slice(w, synth.TID_Q, b, h)[None, None].astype(np.float64) * ds
     k = synth.head_slice(w, synth.TID_K, b, h // w.group)[None, None].astype(np.float64) * ds
     v = synth.head_slice(w, synth.TID_V, b, h // w.group)[None, None].astype(np.float64) * ds
@@ -250,7 +250,8 @@ def run_ours(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
-    fp8 = w.dtype == "e4m3"
+    fp8 = w.dtype in ("e4m3", "e5m2")
+    e5m2 = w.dtype == "e5m2"
     # dense FP8 peak = measured bf16 x the nominal 2x (4.5 vs 2.25 PFLOP/s dense)
     peak_mul = 2.0 if fp8 else 1.0
     peak = float(peaks["bf16_tflops"]) * peak_mul
@@ -264,7 +265,7 @@ def run_ours(args, w, world, rank, local):
     # inputs: generated on the host (seeded), kept pinned for the e2e leg
     host = {}
     tids = (("q", synth.TID_Q), ("k", synth.TID_K), ("v", synth.TID_V)) + ((("do", synth.TID_DO),) if w.backward else ())
-    in_dtype = torch.float8_e4m3fn if fp8 else torch.bfloat16
+    in_dtype = (torch.float8_e5m2 if e5m2 else torch.float8_e4m3fn) if fp8 else torch.bfloat16
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
     share = 1.0
     if args.shard == "heads":
@@ -295,7 +296,7 @@ def run_ours(args, w, world, rank, local):
         if fp8:
             ds = w.descale
             rc = fa.fwd_fp8_raw(P(d_in["q"]), P(d_in["k"]), P(d_in["v"]), ds, ds, ds, P(o), P(lse), B, Hq, Hkv, N, d,
-                                w.causal, w.scale, sp)
+                                w.causal, w.scale, sp, e5m2=e5m2)
         else:
             rc = fa.fwd_raw(P(d_in["q"]), P(d_in["k"]), P(d_in["v"]), P(o), P(lse), B, Hq, Hkv, N, d, w.causal,
                             w.scale, sp)
@@ -390,7 +391,7 @@ def run_ours(args, w, world, rank, local):
             if fp8:
                 ds = w.descale
                 rc = fa.fwd_fp8_raw(P(ins["q"]), P(ins["k"]), P(ins["v"]), ds, ds, ds, P(outs["o"]), P(outs["lse"]),
-                                    B, Hq, Hkv, N, d, w.causal, w.scale, sptr)
+                                    B, Hq, Hkv, N, d, w.causal, w.scale, sptr, e5m2=e5m2)
             else:
                 rc = fa.fwd_raw(P(ins["q"]), P(ins["k"]), P(ins["v"]), P(outs["o"]), P(outs["lse"]), B, Hq, Hkv, N,
                                 d, w.causal, w.scale, sptr)
@@ -696,7 +697,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c3",
-                    help="c2, c3, c3n, c5 (bf16 fwd+bwd), c4, c6 (bf16 fwd), f3, f4 (E4M3 fwd), dec (decode)")
+                    help="c2, c3, c3n, c5 (bf16 fwd+bwd), c4, c6 (bf16 fwd), f3, f4 (E4M3 fwd), f5 (E5M2 fwd), dec (decode)")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N>1: every rank runs the whole workload (weak scaling) or its slice of the heads (strong)")
     ap.add_argument("--e2e-steps", type=int, default=10)

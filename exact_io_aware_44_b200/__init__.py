@@ -34,6 +34,7 @@ SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_fwd_fp8": (_I, [_P, _P, _P, _F, _F, _F, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_fwd_e5m2": (_I, [_P, _P, _P, _F, _F, _F, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "fa_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
@@ -140,21 +141,26 @@ def fwd(q, k, v, causal: bool = True, scale: float | None = None, out=None, lse=
 
 
 def fwd_fp8_raw(q_ptr, k_ptr, v_ptr, descale_q, descale_k, descale_v, o_ptr, lse_ptr, B, Hq, Hkv, N, d, causal,
-                scale, stream_ptr):
-    """fa_fwd_fp8 on raw device pointers (ints); returns the status code."""
-    return lib.fa_fwd_fp8(_P(q_ptr), _P(k_ptr), _P(v_ptr), float(descale_q), float(descale_k), float(descale_v),
-                          _P(o_ptr), _P(lse_ptr), B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _P(stream_ptr))
+                scale, stream_ptr, e5m2=False):
+    """fa_fwd_fp8 (or fa_fwd_e5m2) on raw device pointers (ints); returns the status code."""
+    fn = lib.fa_fwd_e5m2 if e5m2 else lib.fa_fwd_fp8
+    return fn(_P(q_ptr), _P(k_ptr), _P(v_ptr), float(descale_q), float(descale_k), float(descale_v),
+              _P(o_ptr), _P(lse_ptr), B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _P(stream_ptr))
 
 
 def fwd_fp8(q, k, v, descale_q: float, descale_k: float, descale_v: float, causal: bool = True,
             scale: float | None = None, out=None, lse=None, stream=None):
-    """Forward pass on E4M3 inputs (torch.float8_e4m3fn, d = 128) with one descale
-    per tensor: the real inputs are descale_q * q, descale_k * k, descale_v * v.
-    Returns (o, lse) with o in bf16. `scale` defaults to 1/sqrt(d)."""
+    """Forward pass on FP8 inputs (torch.float8_e4m3fn or torch.float8_e5m2, all
+    three the same, d = 128) with one descale per tensor: the real inputs are
+    descale_q * q, descale_k * k, descale_v * v. Returns (o, lse) with o in bf16.
+    `scale` defaults to 1/sqrt(d)."""
     import torch
     B, Hq, Hkv, N, d = _dims(q, k)
+    if q.dtype not in (torch.float8_e4m3fn, torch.float8_e5m2):
+        raise TypeError("q, k, v must be torch.float8_e4m3fn or torch.float8_e5m2")
+    e5m2 = q.dtype == torch.float8_e5m2
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _require(t, n, torch.float8_e4m3fn, q.device)
+        _require(t, n, q.dtype, q.device)
     if v.shape != k.shape:
         raise ValueError("v must have the shape of k")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
@@ -164,8 +170,9 @@ def fwd_fp8(q, k, v, descale_q: float, descale_k: float, descale_v: float, causa
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     _require(out, "out", torch.bfloat16, q.device)
     _require(lse, "lse", torch.float32, q.device)
-    _check(lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), float(descale_q), float(descale_k), float(descale_v), _ptr(out),
-                          _ptr(lse), B, Hq, Hkv, N, d, int(bool(causal)), scale, _stream_ptr(stream)), "fa_fwd_fp8")
+    fn = lib.fa_fwd_e5m2 if e5m2 else lib.fa_fwd_fp8
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), float(descale_q), float(descale_k), float(descale_v), _ptr(out),
+              _ptr(lse), B, Hq, Hkv, N, d, int(bool(causal)), scale, _stream_ptr(stream)), "fa_fwd_fp8")
     return out, lse
 
 

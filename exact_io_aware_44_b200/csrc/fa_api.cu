@@ -168,8 +168,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   return FA_OK;
 }
 
-int fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, float descale_k, float descale_v,
-               void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+static int fwd_f8(bool e5m2, const void* q, const void* k, const void* v, float descale_q, float descale_k,
+                  float descale_v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                  void* stream) {
   bool empty;
   int rc = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
   if (rc != FA_OK) return rc;
@@ -200,8 +201,20 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, flo
   p.scale_log2 = c;
   p.o_scale = descale_v;
   p.wait_budget_ns = g_wait_budget_ns.load();
-  if (launch_fwd_e4m3(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  const cudaError_t e = e5m2 ? launch_fwd_e5m2(tq, tk, tv, p, static_cast<cudaStream_t>(stream))
+                             : launch_fwd_e4m3(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, float descale_k, float descale_v,
+               void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  return fwd_f8(false, q, k, v, descale_q, descale_k, descale_v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream);
+}
+
+int fa_fwd_e5m2(const void* q, const void* k, const void* v, float descale_q, float descale_k, float descale_v,
+                void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  return fwd_f8(true, q, k, v, descale_q, descale_k, descale_v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream);
 }
 
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Hq, int Hkv, int N,

@@ -18,11 +18,11 @@
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 [384,384+d);
 // P_t (bf16 pairs, 64 columns) overwrites the first half of S_t once it is read.
 //
-// E4M3 inputs (d = 128) run the same kernel with kind::f8f6f4 MMAs: a tile is
-// 16 KB (one 128-byte swizzle block wide), the ring holds 10 stages, an MMA
-// steps 32 elements of K, and P is rounded to E4M3, four keys per TMEM column
-// (32 columns). The Q and K descales fold into c; V's descale multiplies the
-// final 1/l.
+// E4M3 or E5M2 inputs (d = 128) run the same kernel with kind::f8f6f4 MMAs: a
+// tile is 16 KB (one 128-byte swizzle block wide), the ring holds 10 stages, an
+// MMA steps 32 elements of K, and P is rounded to the inputs' format, four keys
+// per TMEM column (32 columns), so both operands of every MMA share one type. The
+// Q and K descales fold into c; V's descale multiplies the final 1/l.
 //
 // Per key tile j, a softmax thread loads its row of S_t, applies the causal
 // mask on the diagonal tile, updates the running max, and computes
@@ -67,7 +67,7 @@ constexpr int kPolyPairs = FA_FWD_POLY_PAIRS;
 #endif
 constexpr int kPolyPairs64 = FA_FWD64_POLY_PAIRS;  // the same, for d = 64 (bf16)
 
-// D: head dim; FP8: E4M3 Q, K, V and P (kind::f8f6f4 MMAs), else bf16 (kind::f16).
+// D: head dim; FP8: 8-bit Q, K, V and P (E4M3 or E5M2, kind::f8f6f4 MMAs), else bf16 (kind::f16).
 template <int D, bool FP8>
 struct FwdCfg {
   static constexpr int kElem = FP8 ? 1 : 2;                      // bytes per element
@@ -95,10 +95,32 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int D, bool FP8>
+// Element kinds: bf16 (kind::f16 MMAs), or an 8-bit float for Q, K, V and P
+// (kind::f8f6f4 MMAs with E4M3 or E5M2 in both operands).
+constexpr int kKindBf16 = 0, kKindE4M3 = 1, kKindE5M2 = 2;
+
+// kind::f8f6f4 instruction descriptor with both operand formats set (E4M3 = 0, E5M2 = 1).
+__host__ __device__ constexpr uint32_t idesc_f8_f32(int kind, int M, int N, bool a_mn, bool b_mn) {
+  return idesc_e4m3_f32(M, N, a_mn, b_mn) | ((kind == kKindE5M2 ? 1u : 0u) << 7) |
+         ((kind == kKindE5M2 ? 1u : 0u) << 10);
+}
+// Four fp32 values to E5M2 (round to nearest, saturating), packed low byte first.
+__device__ __forceinline__ uint32_t pack_e5m2x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e5m2x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e5m2x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
+template <int D, int KIND>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  constexpr bool FP8 = KIND != kKindBf16;
   using C = FwdCfg<D, FP8>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -209,8 +231,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     regs_dec<kRegsControl, kRegsLaunch>();
     const bool leader = lane == 0;
     constexpr uint32_t kIdescS =
-        FP8 ? idesc_e4m3_f32(kTileM, kTileN, false, false) : idesc_bf16_f32(kTileM, kTileN, false, false);
-    constexpr uint32_t kIdescPV = FP8 ? idesc_e4m3_f32(kTileM, D, false, true) : idesc_bf16_f32(kTileM, D, false, true);
+        FP8 ? idesc_f8_f32(KIND, kTileM, kTileN, false, false) : idesc_bf16_f32(kTileM, kTileN, false, false);
+    constexpr uint32_t kIdescPV =
+        FP8 ? idesc_f8_f32(KIND, kTileM, D, false, true) : idesc_bf16_f32(kTileM, D, false, true);
     const uint64_t d_q = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
     const uint64_t d_k = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);           // K-major view
     const uint64_t d_v = sdesc_sw128(smem_u32(smem + C::kOffKV), C::kRegion, 1024);   // MN-major view
@@ -382,7 +405,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           rs2[0] = f2_add(rs2[0], f2_pack(e0, e1));
           rs2[1] = f2_add(rs2[1], f2_pack(e2, e3));
           if constexpr (FP8) {
-            pk[i / 4] = pack_e4m3x4(e0, e1, e2, e3);
+            pk[i / 4] = KIND == kKindE5M2 ? pack_e5m2x4(e0, e1, e2, e3) : pack_e4m3x4(e0, e1, e2, e3);
           } else {
             pk[i / 2] = pack_bf16x2(e0, e1);
             pk[i / 2 + 1] = pack_bf16x2(e2, e3);
@@ -455,20 +478,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
-template <int D, bool FP8>
+template <int D, int KIND>
 cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                          cudaStream_t stream) {
-  using C = FwdCfg<D, FP8>;
+  using C = FwdCfg<D, KIND != kKindBf16>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   const long long grid = (long long)p.B * p.Hq * p.n_qblk;
-  fwd_kernel<D, FP8><<<(unsigned)grid, kFwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  fwd_kernel<D, KIND><<<(unsigned)grid, kFwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -476,15 +499,20 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int d, cudaStream_t s) {
-  if (d == 256) return launch_fwd_d<256, false>(tq, tk, tv, p, s);
-  return d == 128 ? launch_fwd_d<128, false>(tq, tk, tv, p, s) : launch_fwd_d<64, false>(tq, tk, tv, p, s);
+  if (d == 256) return launch_fwd_d<256, kKindBf16>(tq, tk, tv, p, s);
+  return d == 128 ? launch_fwd_d<128, kKindBf16>(tq, tk, tv, p, s) : launch_fwd_d<64, kKindBf16>(tq, tk, tv, p, s);
 }
 
 int fwd_tiles_per_cta(int d) { return d == 256 ? FwdCfg<256, false>::kTiles : 2; }
 
 cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, cudaStream_t s) {
-  return launch_fwd_d<128, true>(tq, tk, tv, p, s);
+  return launch_fwd_d<128, kKindE4M3>(tq, tk, tv, p, s);
+}
+
+cudaError_t launch_fwd_e5m2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, cudaStream_t s) {
+  return launch_fwd_d<128, kKindE5M2>(tq, tk, tv, p, s);
 }
 
 }  // namespace fa

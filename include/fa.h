@@ -99,6 +99,16 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, flo
                void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * fa_fwd_e5m2 -- fa_fwd_fp8 with the inputs stored as E5M2 bytes (OCP FP8: 2
+ * mantissa bits, finite max 57344), the page's other FP8 format. Arguments,
+ * layouts and return codes are those of fa_fwd_fp8; P is rounded to E5M2 (values
+ * below 2^-17 of the tile's reference maximum become 0), so both operands of
+ * every MMA are E5M2.
+ */
+int fa_fwd_e5m2(const void* q, const void* k, const void* v, float descale_q, float descale_k, float descale_v,
+                void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
+
+/*
  * fa_decode_workspace_bytes -- device scratch that fa_decode needs.
  *
  * Per key split, a float32 partial output [B*Hq*Nq, d] and a float32 partial

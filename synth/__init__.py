@@ -26,6 +26,7 @@ Workloads (shapes from the pages' long-context regime; all synthetic, no dataset
   c6  bf16 fwd,  B=2 H=16 N=8192 d=256, causal
   f3  E4M3 fwd,  B=2 H=32 N=8192 d=128, causal, std 1/sqrt(2) (c3's shape)
   f4  E4M3 fwd,  B=1 H=16 N=65536 d=128, causal (c4's shape)
+  f5  E5M2 fwd,  c3's shape
   dec decode,    B=16 Hq=32 Hkv=8, Nq=1 new query against Nk=32768 cached keys, d=128
 """
 from __future__ import annotations
@@ -50,7 +51,7 @@ class Workload:
     N: int
     d: int
     causal: bool
-    dtype: str  # "f32", "bf16" or "e4m3"
+    dtype: str  # "f32", "bf16", "e4m3" or "e5m2"
     backward: bool
     seed: int
     std: float = 1.0
@@ -70,8 +71,10 @@ class Workload:
 
     @property
     def descale(self) -> float:
-        """E4M3 workloads: the float32 value that multiplies every stored code."""
-        return float(np.float32(8.0 * self.std / 448.0))
+        """FP8 workloads: the float32 value that multiplies every stored code
+        (8 standard deviations map to the format's largest finite value)."""
+        top = E5M2_MAX if self.dtype == "e5m2" else E4M3_MAX
+        return float(np.float32(8.0 * self.std / top))
 
     def fwd_flops(self) -> float:
         f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
@@ -102,11 +105,33 @@ WORKLOADS = {
     "f3": Workload("f3", 2, 32, 32, 8192, 128, True, "e4m3", False, 1006,
                    std=1.0 / math.sqrt(2.0),
                    sample_heads=((0, 0), (0, 17), (1, 6), (1, 31)), sample_rows=256),
+    "f5": Workload("f5", 2, 32, 32, 8192, 128, True, "e5m2", False, 1011,
+                   std=1.0 / math.sqrt(2.0),
+                   sample_heads=((0, 0), (0, 17), (1, 6), (1, 31)), sample_rows=256),
     "f4": Workload("f4", 1, 16, 16, 65536, 128, True, "e4m3", False, 1007,
                    sample_heads=((0, 0), (0, 5), (0, 10), (0, 15)), sample_rows=256),
 }
 
 E4M3_MAX = 448.0
+E5M2_MAX = 57344.0
+
+
+def _round_to_fp8(x: np.ndarray, mant_bits: int, min_exp: int, top: float) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32).astype(np.float64)
+    a = np.minimum(np.abs(x), top)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, float(min_exp))    # below the smallest normal the step stays (subnormals)
+    step = np.exp2(e - mant_bits)
+    r = np.minimum(np.round(a / step) * step, top)   # numpy rounds halves to even
+    return (np.sign(x) * r).astype(np.float32)
+
+
+def round_to_e5m2(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest E5M2 value (OCP FP8: 2 mantissa bits,
+    exponent bias 15, subnormal step 2^-16), ties to even, saturating at +-57344.
+    Returns float32."""
+    return _round_to_fp8(x, 2, -14, E5M2_MAX)
 
 
 def round_to_e4m3(x: np.ndarray) -> np.ndarray:
@@ -157,6 +182,8 @@ def head_slice(w: Workload, tid: int, b: int, h: int, n: int | None = None) -> n
         x = round_to_bf16(x)
     elif w.dtype == "e4m3":
         x = round_to_e4m3(x / np.float32(w.descale))
+    elif w.dtype == "e5m2":
+        x = round_to_e5m2(x / np.float32(w.descale))
     return x
 
 

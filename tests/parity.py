@@ -6,8 +6,9 @@ bf16-rounded inputs, so input quantisation is not counted):
   forward   max |dO| <= 2e-2, mean |dO| <= 2e-3, max |dLSE| <= 1e-3
   backward  relative Frobenius error <= 1e-2 for each of dQ, dK, dV
 
-E4M3 forward (the oracle runs on the dequantised E4M3 inputs, so again only the
-kernel's own rounding counts). S is exact E4M3 products summed in fp32, so LSE
+FP8 forward (the oracle runs on the dequantised E4M3 or E5M2 inputs, so again only
+the kernel's own rounding counts; the figures below are E4M3's, E5M2 has 2^-3 relative
+and 2^-17 absolute in place of 2^-4 and 2^-10). S is exact E4M3 products summed in fp32, so LSE
 keeps the 1e-3 bound. The one coarse step is P: the kernel rounds
 e_j = exp(s_j - m_ref) (m_ref <= the row max) to E4M3 before P V but divides by
 L = sum_j e_j unrounded. E4M3 rounding moves e by at most 2^-4 e (normal range)
@@ -58,14 +59,23 @@ def rel_fro(x, ref):
     return float(np.linalg.norm(np.asarray(x, np.float64) - ref) / den)
 
 
-def e4m3_step(e):
-    """Spacing of E4M3 values around e >= 0 (2^-9 in the subnormal range)."""
+# FP8 formats: mantissa bits and the smallest normal exponent
+FP8_FORMATS = {"e4m3": (3, -6), "e5m2": (2, -14)}
+
+
+def fp8_step(e, fmt="e4m3"):
+    """Spacing of the format's values around e >= 0 (constant in the subnormal range)."""
+    mant, emin = FP8_FORMATS[fmt]
     e = np.asarray(e, np.float64)
     ex = np.floor(np.log2(np.where(e > 0, e, 1.0)))
-    return np.exp2(np.maximum(ex, -6.0) - 3.0)
+    return np.exp2(np.maximum(ex, float(emin)) - mant)
 
 
-def fp8_fwd_model(p_rows, v, o_ref):
+def e4m3_step(e):
+    return fp8_step(e, "e4m3")
+
+
+def fp8_fwd_model(p_rows, v, o_ref, fmt="e4m3"):
     """Per-element error bound and the modelled mean |dO| for the E4M3 forward.
 
     p_rows [R, N]: exact softmax rows (oracle.head_probs64); v [N, d] the
@@ -76,20 +86,22 @@ def fp8_fwd_model(p_rows, v, o_ref):
     pmax = p.max(axis=1)
     n = (p > 0).sum(axis=1)
     vmax = np.abs(v).max(axis=0)
-    bound = (2.0 ** -4) * (p @ np.abs(v)) + (2.0 ** -10) * (n * pmax)[:, None] * vmax[None, :] \
+    mant, emin = FP8_FORMATS[fmt]
+    rel, flush = 2.0 ** -(mant + 1), 2.0 ** (emin - mant - 1)   # half a step: relative, and absolute below normals
+    bound = rel * (p @ np.abs(v)) + flush * (n * pmax)[:, None] * vmax[None, :] \
         + (2.0 ** -8) * np.abs(o_ref) + 1e-5
     e = p / pmax[:, None]                                   # kernel units with m_ref = row max
-    var_unit = np.where(e >= 2.0 ** -10, e4m3_step(e) ** 2 / 12.0, e * e)
+    var_unit = np.where(e >= flush, fp8_step(e, fmt) ** 2 / 12.0, e * e)
     sigma = np.sqrt(var_unit @ (v * v)) * pmax[:, None]     # divided by L = 1 / pmax
     mean = 1.1 * float(sigma.mean()) + (2.0 ** -9) * float(np.abs(o_ref).mean()) + 1e-6
     return bound, mean
 
 
-def assert_fp8_fwd_ok(o_gpu, lse_gpu, o_ref, lse_ref, p_rows, v, label=""):
+def assert_fp8_fwd_ok(o_gpu, lse_gpu, o_ref, lse_ref, p_rows, v, label="", fmt="e4m3"):
     """o_gpu, o_ref, p_rows: rows of ONE head; v [N, d] that head's dequantised V."""
     o_gpu = np.asarray(o_gpu, np.float64)
     err = np.abs(o_gpu - o_ref)
-    bound, mean = fp8_fwd_model(p_rows, v, o_ref)
+    bound, mean = fp8_fwd_model(p_rows, v, o_ref, fmt)
     worst = float((err / bound).max()) if err.size else 0.0
     dl = float(np.abs(np.asarray(lse_gpu, np.float64) - lse_ref).max()) if err.size else 0.0
     stats = {"max_abs_o": float(err.max()) if err.size else 0.0, "mean_abs_o": float(err.mean()) if err.size else 0.0,

@@ -1,4 +1,4 @@
-"""E4M3 forward parity: fa_fwd_fp8 against the float64 oracle run on the
+"""FP8 forward parity (fa_fwd_fp8 with E4M3 inputs, fa_fwd_e5m2 with E5M2): against the float64 oracle run on the
 dequantised inputs (code * descale), with the error model of tests/parity.py:
 every output element within its rounding bound, the mean error within the
 modelled mean, and LSE within 1e-3.
@@ -15,20 +15,25 @@ from tests.parity import assert_fp8_fwd_ok, to_dev
 pytestmark = pytest.mark.gpu
 
 
-def e4m3_dev(codes, device):
+def fp8_dev(codes, device, fmt="e4m3"):
     import torch
-    return torch.from_numpy(np.ascontiguousarray(codes, np.float32)).to(torch.float8_e4m3fn).to(device)
+    dt = torch.float8_e5m2 if fmt == "e5m2" else torch.float8_e4m3fn
+    return torch.from_numpy(np.ascontiguousarray(codes, np.float32)).to(dt).to(device)
 
 
-def run_fp8(qc, kc, vc, dq, dk, dv, causal, scale, device):
+def e4m3_dev(codes, device):
+    return fp8_dev(codes, device, "e4m3")
+
+
+def run_fp8(qc, kc, vc, dq, dk, dv, causal, scale, device, fmt="e4m3"):
     import exact_io_aware_44_b200 as fa
-    o, lse = fa.fwd_fp8(e4m3_dev(qc, device), e4m3_dev(kc, device), e4m3_dev(vc, device), dq, dk, dv,
+    o, lse = fa.fwd_fp8(fp8_dev(qc, device, fmt), fp8_dev(kc, device, fmt), fp8_dev(vc, device, fmt), dq, dk, dv,
                         causal=causal, scale=scale)
     assert fa.get_status() == 0
     return o.float().cpu().numpy(), lse.cpu().numpy()
 
 
-def check_heads(qc, kc, vc, dq, dk, dv, causal, scale, o, lse, heads=None, rows_of=None, label=""):
+def check_heads(qc, kc, vc, dq, dk, dv, causal, scale, o, lse, heads=None, rows_of=None, label="", fmt="e4m3"):
     """Compare the given (b, h) heads (all by default), each on `rows_of(b, h)` rows (all by default)."""
     B, Hq, N, _ = qc.shape
     g = Hq // kc.shape[1]
@@ -41,7 +46,7 @@ def check_heads(qc, kc, vc, dq, dk, dv, causal, scale, o, lse, heads=None, rows_
         v64 = vc[b, h // g].astype(np.float64) * dv
         o_ref, lse_ref = oracle.head_fwd64(q64, k64, v64, causal, scale, rows=rows)
         p = oracle.head_probs64(q64, k64, causal, scale, rows=rows)
-        st = assert_fp8_fwd_ok(o[b, h, rows], lse[b, h, rows], o_ref, lse_ref, p, v64, f"{label} head {(b, h)}")
+        st = assert_fp8_fwd_ok(o[b, h, rows], lse[b, h, rows], o_ref, lse_ref, p, v64, f"{label} head {(b, h)}", fmt)
         for key, val in st.items():
             worst[key] = max(worst.get(key, 0.0), val)
     return worst
@@ -51,8 +56,8 @@ def check_workload(w, device, causal=None):
     causal = w.causal if causal is None else causal
     qc, kc, vc = (synth.tensor(w, t) for t in (synth.TID_Q, synth.TID_K, synth.TID_V))
     ds = w.descale
-    o, lse = run_fp8(qc, kc, vc, ds, ds, ds, causal, w.scale, device)
-    return check_heads(qc, kc, vc, ds, ds, ds, causal, w.scale, o, lse, label=w.name)
+    o, lse = run_fp8(qc, kc, vc, ds, ds, ds, causal, w.scale, device, w.dtype)
+    return check_heads(qc, kc, vc, ds, ds, ds, causal, w.scale, o, lse, label=w.name, fmt=w.dtype)
 
 
 SHAPES = [
@@ -142,3 +147,36 @@ def test_fp8_fwd_full_size_sampled(cuda_device, name):
     o, lse = run_fp8(qc, kc, vc, ds, ds, ds, w.causal, w.scale, cuda_device)
     check_heads(qc, kc, vc, ds, ds, ds, w.causal, w.scale, o, lse, heads=list(w.sample_heads),
                 rows_of=lambda b, h: synth.sample_rows(w, b, h), label=w.name)
+
+
+# ------------------------------------------------------------------ E5M2 (fa_fwd_e5m2)
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_e5m2_fwd_small(cuda_device, shape, causal):
+    B, Hq, Hkv, N = shape
+    w = synth.small(B, Hq, Hkv, N, 128, causal, seed=700 + N, dtype="e5m2")
+    check_workload(w, cuda_device)
+
+
+def test_e5m2_fwd_distinct_descales_and_rescales(cuda_device):
+    """Different descales per tensor and keys whose scores grow along the sequence."""
+    rng = np.random.default_rng(41)
+    N, d = 1100, 128
+    qc = synth.round_to_e5m2(np.abs(rng.standard_normal((1, 2, N, d))).astype(np.float32) * 3000)
+    ramp = np.linspace(0.2, 3.0, N, dtype=np.float32)[:, None]
+    kc = synth.round_to_e5m2((np.abs(rng.standard_normal((1, 1, N, d))) * ramp * 2000).astype(np.float32))
+    vc = synth.round_to_e5m2(rng.standard_normal((1, 1, N, d)).astype(np.float32) * 5000)
+    dq, dk, dv = 3.1e-4, 4.7e-4, 1.3e-4
+    for causal in (True, False):
+        o, lse = run_fp8(qc, kc, vc, dq, dk, dv, causal, 1 / math.sqrt(d), cuda_device, "e5m2")
+        check_heads(qc, kc, vc, dq, dk, dv, causal, 1 / math.sqrt(d), o, lse, label=f"e5m2 {causal}", fmt="e5m2")
+
+
+def test_e5m2_fwd_full_size_sampled(cuda_device):
+    w = synth.WORKLOADS["f5"]
+    qc, kc, vc = (synth.tensor(w, t) for t in (synth.TID_Q, synth.TID_K, synth.TID_V))
+    ds = w.descale
+    o, lse = run_fp8(qc, kc, vc, ds, ds, ds, w.causal, w.scale, cuda_device, "e5m2")
+    check_heads(qc, kc, vc, ds, ds, ds, w.causal, w.scale, o, lse, heads=list(w.sample_heads),
+                rows_of=lambda b, h: synth.sample_rows(w, b, h), label=w.name, fmt="e5m2")

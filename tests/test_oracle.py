@@ -381,6 +381,17 @@ def test_synth_e4m3_rounding_matches_torch():
     assert synth.round_to_e4m3(np.float32([-1e6]))[0] == -448.0
 
 
+def test_synth_e5m2_rounding_matches_torch():
+    import torch
+    x = np.random.default_rng(7).standard_normal(20000).astype(np.float32)
+    x *= np.repeat(np.float32([1e-5, 0.05, 1.0, 5000.0]), 5000)
+    x[:6] = [2.0 ** -17, 3 * 2.0 ** -18, 1.125, 1.375, 57344.0, -50000.0]  # ties (to even) and the top
+    ours = synth.round_to_e5m2(x)
+    ref = torch.from_numpy(x).to(torch.float8_e5m2).to(torch.float32).numpy()
+    assert np.array_equal(ours, ref)
+    assert synth.round_to_e5m2(np.float32([1e6]))[0] == 57344.0   # saturates
+
+
 def test_synth_e4m3_workload_codes():
     w = synth.WORKLOADS["f3"]
     x = synth.head_slice(w, synth.TID_K, 1, 5, n=2048)
