@@ -276,7 +276,7 @@ int check_decode(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, floa
   if (rc != FA_OK) return rc;
   if (Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
   if (causal && Nq > Nk) return FA_ERR_INVALID_ARG;
-  if (d != 128 || (Hq / Hkv) * Nq > 16) return FA_ERR_UNSUPPORTED;
+  if (d != 128 || (long long)(Hq / Hkv) * Nq > 32) return FA_ERR_UNSUPPORTED;
   if ((long long)B * Hkv * (long long)Nk >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
@@ -309,7 +309,7 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   const DecodeSplit sp = decode_split(B, Hkv, Nk, num_splits);
   const long long rows = (long long)B * Hq * Nq;
   CUtensorMap tq, tk, tv;
-  if ((rc = make_map(&tq, q, d, (int)rows, 1, 16)) != FA_OK) return rc;
+  if ((rc = make_map(&tq, q, d, (int)rows, 1, decode_rows_per_cta((Hq / Hkv) * Nq))) != FA_OK) return rc;
   if ((rc = make_map(&tk, k, d, Nk, B * Hkv)) != FA_OK) return rc;
   if ((rc = make_map(&tv, v, d, Nk, B * Hkv)) != FA_OK) return rc;
   DecodeParams p;

@@ -6,7 +6,7 @@
 // ("FlashAttention Kernel & Online Softmax" card: the relation to the KV cache
 // and the decode bandwidth bottleneck). So the design goal is to read K and V
 // exactly once at full bandwidth: one CTA handles all query rows of one GQA
-// group (g query heads x Nq queries, at most 16 rows) against one slice of the
+// group (g query heads x Nq queries, at most 32 rows) against one slice of the
 // keys, and enough slices run side by side to fill the GPU.
 //
 // Each split produces an unnormalised-then-normalised partial output O_s and its
@@ -17,20 +17,21 @@
 // decode_split_kernel (192 threads, d = 128):
 //   warp 0      TMA producer: the group's query rows once, then K and V chunks of
 //               128 keys through a 3-stage ring.
-//   warp 1      allocates TMEM (64 columns); lane 0 issues the MMAs:
-//                 S^T(c) = K_c Q^T   M = 128 keys, N = 16 query rows, K = d -> TMEM
-//                 O^T   += V_c^T P^T  M = d = 128, N = 16, K = 128 keys     -> TMEM
+//   warp 1      allocates TMEM (64 or 128 columns); lane 0 issues the MMAs:
+//                 S^T(c) = K_c Q^T   M = 128 keys, N = R query rows, K = d -> TMEM
+//                 O^T   += V_c^T P^T  M = d = 128, N = R, K = 128 keys      -> TMEM
 //               so keys, and then head-dim columns, sit in TMEM lanes and the few
 //               query rows are the MMA's N (tcgen05 needs M >= 64, N may be 16).
 //   warps 2-5   thread = TMEM lane: key row of S^T, head-dim row of O^T.
-// Per chunk a thread loads its 16 scores, and the CTA keeps one reference max per
+// The kernel is instantiated for R = 16 and R = 32 query rows (the host takes the
+// smaller that holds the group). Per chunk a thread loads its R scores, and the CTA keeps one reference max per
 // query row, raised only when some score exceeds it by more than 2^8 (the exact
 // column max is then reduced across the 128 threads and O^T and the per-thread
 // partial denominators are rescaled); otherwise P = 2^(S c - m_ref) directly.
 // P^T goes to shared memory as the MMA's B operand (K-major, 128-byte swizzle).
 // The denominators are per-thread partial sums, reduced once at the end.
 //
-// TMEM columns: S^T buffers [0,16) and [16,32) (chunk parity), O^T [32,48).
+// TMEM columns: S^T buffers [0,R) and [R,2R) (chunk parity), O^T [2R,3R).
 #include <math.h>
 
 #include "fa.h"
@@ -41,29 +42,32 @@ namespace fa {
 namespace {
 
 constexpr int kDecThreads = 192;
-constexpr int kDecRows = 16;     // query rows per CTA (the MMA N)
 constexpr int kDecChunk = 128;   // keys per chunk (the MMA M)
 constexpr int kDecStages = 3;
 constexpr uint32_t kDecRescaleLog2 = 8;
 
+// R: query rows per CTA (the MMA N: 16 or 32).
+template <int R>
 struct DecCfg {
   static constexpr int D = 128;
   static constexpr int kKV = kDecChunk * D * 2;          // one K or V chunk (32 KB)
   static constexpr int kRegion = kDecChunk * 128;        // 64-column block of a chunk (16 KB)
-  static constexpr int kQRegion = kDecRows * 128;        // 64-column block of the query tile (2 KB)
-  static constexpr int kPRegion = kDecRows * 128;        // 64-key block of a P^T tile (2 KB)
+  static constexpr int kQRegion = R * 128;               // 64-column block of the query tile
+  static constexpr int kPRegion = R * 128;               // 64-key block of a P^T tile
   static constexpr int kOffQ = 0;                        // 2 blocks
   static constexpr int kOffP = kOffQ + 2 * kQRegion;     // 2 buffers x 2 blocks
   static constexpr int kOffKV = kOffP + 4 * kPRegion;    // stages of K then V
-  static constexpr int kOffRed = kOffKV + kDecStages * 2 * kKV;   // [3][4][16] floats, then flags [2][4]
-  static constexpr int kOffBar = kOffRed + 3 * 4 * 16 * 4 + 64;
+  static constexpr int kOffRed = kOffKV + kDecStages * 2 * kKV;   // [3][4][R] floats, then flags [2][4]
+  static constexpr int kOffBar = kOffRed + 3 * 4 * R * 4 + 64;
   // q_full, kv_full[3], kv_empty[3], s_full[2], p_full[2], pv_done[2], vote[2], red_bar, mma_done
   static constexpr int kNumBars = 17;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static_assert(kOffKV % 1024 == 0 && kOffP % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static constexpr int kColS = 0, kColO = 32;
+  // TMEM: S^T buffers [0, R) and [R, 2R) (chunk parity), O^T [2R, 3R)
+  static constexpr int kColS = 0, kColO = 2 * R;
+  static constexpr int kTmemCols = R == 16 ? 64 : 128;
 };
 
 __device__ __forceinline__ uint8_t* align1024d(uint8_t* p) {
@@ -95,6 +99,24 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
+// R-column forms (R = 16 or 32).
+template <int R>
+__device__ __forceinline__ void tmem_ld_r(uint32_t taddr, uint32_t (&r)[R]) {
+  if constexpr (R == 16) {
+    tmem_ld16(taddr, r);
+    tmem_ld_wait16(r);
+  } else {
+    tmem_ld32(taddr, r);
+    tmem_ld_wait(r);
+  }
+}
+template <int R>
+__device__ __forceinline__ void tmem_st_r(uint32_t taddr, const uint32_t (&r)[R]) {
+  if constexpr (R == 16)
+    tmem_st16(taddr, r);
+  else
+    tmem_st32(taddr, r);
+}
 __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
@@ -114,10 +136,12 @@ __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, const
   return ok;
 }
 
+template <int R>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
-  using C = DecCfg;
+  using C = DecCfg<R>;
+  constexpr int kDecRows = R;
   constexpr int S = kDecStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024d(smem_raw);
@@ -131,9 +155,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint64_t* vote_bar = bars + 13;
   uint64_t* red_bar = bars + 15;
   uint64_t* mma_done = bars + 16;
-  // [3][4][16]: column maxima by chunk parity, then the final denominators
+  // [3][4][R]: column maxima by chunk parity, then the final denominators
   float* red = reinterpret_cast<float*>(smem + C::kOffRed);
-  volatile int* flags = reinterpret_cast<volatile int*>(smem + C::kOffRed + 3 * 4 * 16 * 4);  // [2][4]
+  volatile int* flags = reinterpret_cast<volatile int*>(smem + C::kOffRed + 3 * 4 * R * 4);  // [2][4]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -144,7 +168,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int b = bkv / p.Hkv;
   const int kvh = bkv % p.Hkv;
   const int g = p.Hq / p.Hkv;
-  const int rows = g * p.Nq;                                 // valid query rows (<= 16)
+  const int rows = g * p.Nq;                                 // valid query rows (<= R)
   const int row0 = (b * p.Hq + kvh * g) * p.Nq;              // first global query row
   const int n_chunks_all = (p.Nk + kDecChunk - 1) / kDecChunk;
   const int c_begin = min(split * p.chunks_per_split, n_chunks_all);
@@ -170,7 +194,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 64);
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -225,7 +249,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const uint32_t ao = (k >> 2) * C::kRegion + (k & 3) * 32;
         const uint32_t bo = (k >> 2) * C::kQRegion + (k & 3) * 32;
         if (leader)
-          mma_bf16_ss(tmem + C::kColS + (c & 1) * 16, desc_advance(a0, ao), desc_advance(d_q, bo), kIdS,
+          mma_bf16_ss(tmem + C::kColS + (c & 1) * R, desc_advance(a0, ao), desc_advance(d_q, bo), kIdS,
                       k > 0 ? 1u : 0u);
       }
       if (leader) mma_commit(&s_full[c & 1]);
@@ -277,29 +301,34 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float c2 = p.scale_log2;
     float m_ref[kDecRows], l_part[kDecRows];
-    int last_key[kDecRows];  // causal: the last key each query row may see (-1: row unused)
 #pragma unroll
     for (int j = 0; j < kDecRows; ++j) {
       m_ref[j] = -INFINITY;
       l_part[j] = 0.f;
-      const int i = j % p.Nq;
-      last_key[j] = j < rows ? (p.causal ? p.Nk - p.Nq + i : p.Nk - 1) : -1;
     }
+    // Row j is query i = j mod Nq of its head; with the causal mask it sees keys up to
+    // Nk - Nq + i. Keys up to all_vis are seen by every valid row.
+    const uint32_t row_mask = rows >= 32 ? 0xffffffffu : ((1u << rows) - 1u);
+    const int all_vis = p.causal ? p.Nk - p.Nq : p.Nk - 1;
     uint32_t vote_ph[2] = {0, 0}, red_ph = 0;
     bool ok = true;
     for (int c = 0; c < n && ok; ++c) {
       if (!(ok = warp_wait(&s_full[c & 1], (c >> 1) & 1, w))) break;
       tc_fence_after();
-      uint32_t r[16];
-      tmem_ld16(tmem + lane_off + C::kColS + (c & 1) * 16, r);
-      tmem_ld_wait16(r);
+      uint32_t r[R];
+      tmem_ld_r<R>(tmem + lane_off + C::kColS + (c & 1) * R, r);
       const int key = (c_begin + c) * kDecChunk + t;
+      uint32_t vis = key < k_end ? row_mask : 0u;  // bit j: row j sees this key
+      if (key < k_end && key > all_vis) {           // the causal edge, in the last chunk only
+        vis = 0u;
+        for (int j = 0; j < rows; ++j)
+          if (key <= p.Nk - p.Nq + j % p.Nq) vis |= 1u << j;
+      }
       float x[kDecRows];
       bool over = false;
 #pragma unroll
       for (int j = 0; j < kDecRows; ++j) {
-        const bool vis = key < k_end && key <= last_key[j];
-        x[j] = vis ? __uint_as_float(r[j]) * c2 : -INFINITY;
+        x[j] = (vis >> j) & 1u ? __uint_as_float(r[j]) * c2 : -INFINITY;
         over |= x[j] > m_ref[j] + (float)kDecRescaleLog2;
       }
       // does any thread need a higher reference max for some row?
@@ -310,19 +339,19 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                            flags[(c & 1) * 4 + 3];
       if (rescale) {
         // exact column max of this chunk over the 128 threads
-        float* rd = red + (c & 1) * 64;
+        float* rd = red + (c & 1) * 4 * R;
 #pragma unroll
         for (int j = 0; j < kDecRows; ++j) {
           float v = x[j];
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == 0) rd[wq * 16 + j] = v;
+          if (lane == 0) rd[wq * R + j] = v;
         }
         if (!(ok = group_sync(red_bar, red_ph, w))) break;
         float alpha[kDecRows];
 #pragma unroll
         for (int j = 0; j < kDecRows; ++j) {
-          const float cm = fmaxf(fmaxf(rd[j], rd[16 + j]), fmaxf(rd[32 + j], rd[48 + j]));
+          const float cm = fmaxf(fmaxf(rd[j], rd[R + j]), fmaxf(rd[2 * R + j], rd[3 * R + j]));
           const float m_new = fmaxf(m_ref[j], cm);
           alpha[j] = (m_new == -INFINITY || m_ref[j] == m_new) ? 1.f : ex2(m_ref[j] - m_new);
           m_ref[j] = m_new;
@@ -332,12 +361,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (c > 0) {
           if (!(ok = warp_wait(&pv_done[(c - 1) & 1], ((c - 1) >> 1) & 1, w))) break;
           tc_fence_after();
-          uint32_t o[16];
-          tmem_ld16(tmem + lane_off + C::kColO, o);
-          tmem_ld_wait16(o);
+          uint32_t o[R];
+          tmem_ld_r<R>(tmem + lane_off + C::kColO, o);
 #pragma unroll
           for (int j = 0; j < kDecRows; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha[j]);
-          tmem_st16(tmem + lane_off + C::kColO, o);
+          tmem_st_r<R>(tmem + lane_off + C::kColO, o);
           tmem_st_wait();
         }
       }
@@ -360,26 +388,25 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     // epilogue: denominators reduced over the 128 threads, O^T / l -> partial outputs
     if (ok && n > 0) {
-      float* rd = red + 2 * 64;  // its own slot: a slower thread may still read the last maxima
+      float* rd = red + 2 * 4 * R;  // its own slot: a slower thread may still read the last maxima
 #pragma unroll
       for (int j = 0; j < kDecRows; ++j) {
         float v = l_part[j];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) rd[wq * 16 + j] = v;
+        if (lane == 0) rd[wq * R + j] = v;
       }
       ok = group_sync(red_bar, red_ph, w);
       if (ok) ok = warp_wait(mma_done, 0, w);
       if (ok) {
         tc_fence_after();
-        uint32_t o[16];
-        tmem_ld16(tmem + lane_off + C::kColO, o);
-        tmem_ld_wait16(o);
+        uint32_t o[R];
+        tmem_ld_r<R>(tmem + lane_off + C::kColO, o);
         float* opart = p.o_part + (size_t)split * p.rows_total * C::D;
 #pragma unroll
         for (int j = 0; j < kDecRows; ++j) {
           if (j < rows) {
-            const float l = rd[j] + rd[16 + j] + rd[32 + j] + rd[48 + j];
+            const float l = rd[j] + rd[R + j] + rd[2 * R + j] + rd[3 * R + j];
             const float inv = l > 0.f ? 1.f / l : 0.f;
             opart[(size_t)(row0 + j) * C::D + t] = __uint_as_float(o[j]) * inv;
             if (t == 0)
@@ -400,7 +427,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -425,22 +452,31 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
 
 }  // namespace
 
-cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
-                          cudaStream_t s) {
-  using C = DecCfg;
+template <int R>
+cudaError_t launch_decode_r(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const DecodeParams& p, cudaStream_t s) {
+  using C = DecCfg<R>;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   dim3 grid((unsigned)p.n_splits, (unsigned)(p.B * p.Hkv));
-  decode_split_kernel<<<grid, kDecThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
+  decode_split_kernel<R><<<grid, kDecThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<(unsigned)p.rows_total, 128, 0, s>>>(p);
   return cudaGetLastError();
+}
+
+int decode_rows_per_cta(int rows) { return rows <= 16 ? 16 : 32; }
+
+cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                          cudaStream_t s) {
+  const int rows = (p.Hq / p.Hkv) * p.Nq;
+  return decode_rows_per_cta(rows) == 16 ? launch_decode_r<16>(tq, tk, tv, p, s) : launch_decode_r<32>(tq, tk, tv, p, s);
 }
 
 }  // namespace fa

@@ -71,6 +71,8 @@ cudaError_t launch_fwd_e5m2(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const FwdParams& p, cudaStream_t s);
 cudaError_t launch_fwd_f32(const FwdF32Params& p, cudaStream_t s);
 // Decode: the split kernel, then the merge of the splits.
+// Query rows per decode CTA for a GQA group of `rows` rows (16 or 32).
+int decode_rows_per_cta(int rows);
 cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           cudaStream_t s);
 // Query rows per tile of the main backward kernel for head dim d (its TMA box height).

@@ -136,7 +136,7 @@ size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, 
  *               device memory, 256-byte aligned, contents on entry irrelevant
  *   num_splits  key splits (<= 0: chosen from the sizes; capped by the number of
  *               128-key chunks)
- *   d must be 128 and (Hq / Hkv) * Nq at most 16 (one CTA serves a whole GQA
+ *   d must be 128 and (Hq / Hkv) * Nq at most 32 (one CTA serves a whole GQA
  *   group's query rows), else FA_ERR_UNSUPPORTED; causal with Nq > Nk is
  *   FA_ERR_INVALID_ARG. Arithmetic: bf16 operands, fp32 accumulation; P is
  *   rounded to bf16 before the P V product; the partials stay fp32.

@@ -87,8 +87,9 @@ def _dec(B=1, Hq=8, Hkv=1, Nq=1, Nk=1000, d=128, causal=1, scale=0.088, splits=0
 
 def test_decode_rejects_bad_arguments_on_host():
     assert _dec(d=64) == -2                        # d = 128 only
-    assert _dec(Hq=32, Hkv=1) == -2                # 32 query rows per group > 16
-    assert _dec(Hq=8, Nq=3) == -2                  # 24 rows > 16
+    assert _dec(Hq=64, Hkv=1) == -2                # 64 query rows per group > 32
+    assert _dec(Hq=8, Nq=5) == -2                  # 40 rows > 32
+    assert _dec(Hq=16, Nq=3) == -2                 # 48 rows > 32
     assert _dec(Nq=5, Nk=4) == -1                  # causal needs Nq <= Nk
     assert _dec(Nk=0) == -1
     assert _dec(Hq=6, Hkv=4) == -1

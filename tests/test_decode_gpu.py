@@ -44,6 +44,11 @@ SHAPES = [
     (2, 16, 1, 1, 3000),    # a 16-head group
     (1, 2, 2, 3, 333),      # no GQA, 3 new tokens
     (1, 4, 4, 2, 4097),
+    (1, 8, 1, 3, 900),      # 24 rows: the 32-row kernel, 8 rows unused
+    (2, 32, 4, 4, 2500),    # GQA group 8 x 4 new tokens = 32 rows
+    (1, 32, 1, 1, 513),     # a 32-head group
+    (1, 2, 1, 16, 640),     # 16 new tokens per head, 32 rows, the causal edge spans 16 keys
+    (1, 1, 1, 17, 17),      # square, 17 rows
 ]
 
 
