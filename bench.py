@@ -49,7 +49,8 @@ NCU_TRAFFIC = {
     # profiles/bwd_main_d128_B2H32N8192_causal.md
     ("bwd_main", "c3"): {"bytes_per_launch": 809986560 + 491049984, "csrc_sha": "7497d3bd4abc43c9"},
     # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md
-    ("decode_split", "dec"): {"bytes_per_launch": 2147724544 + 4109568, "csrc_sha": "812f00ecc35581b6"},
+    ("decode_split", "dec"): {"bytes_per_launch": 2148443904 + 3871232, "csrc_sha": "c1652c60e81fafd1"},
+    ("decode_split", "dec4"): {"bytes_per_launch": 1074819072 + 5263104, "csrc_sha": "c1652c60e81fafd1"},
 }
 
 
@@ -697,7 +698,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c3",
-                    help="c2, c3, c3n, c5 (bf16 fwd+bwd), c4, c6 (bf16 fwd), f3, f4 (E4M3 fwd), f5 (E5M2 fwd), dec (decode)")
+                    help="c2, c3, c3n, c5 (bf16 fwd+bwd), c4, c6 (bf16 fwd), f3, f4 (E4M3 fwd), f5 (E5M2 fwd), dec, dec4 (decode)")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N>1: every rank runs the whole workload (weak scaling) or its slice of the heads (strong)")
     ap.add_argument("--e2e-steps", type=int, default=10)

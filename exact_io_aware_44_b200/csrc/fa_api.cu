@@ -250,24 +250,26 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
 namespace fa {
 namespace {
 
-// Key splits for decode: enough (batch, kv head, split) CTAs for two per SM of a
-// 148-SM part, at most one split per 128-key chunk, and no empty split. A fixed
-// rule (not the current device's SM count) so that the workspace size can be
-// computed without a device.
-constexpr int kDecodeTargetCtas = 296;
-constexpr int kDecodeMaxSplits = 256;
+// Decode work split: all groups' 128-key chunks laid end to end and cut into
+// n_ctas equal slices, one per split-kernel CTA. Automatic: one CTA per SM of a
+// 148-SM part (the kernel keeps one CTA per SM), so the slices run as one wave;
+// num_splits > 0: B * Hkv * num_splits CTAs. Never more CTAs than chunks. A fixed
+// rule of the sizes, not of the current device, so that the workspace size can be
+// computed without one. A slice may cross group boundaries; each (group, CTA)
+// piece is a segment with its own slot (group + CTA index) in the workspace.
+constexpr int kDecodeSms = 148;
 
 struct DecodeSplit {
-  int n_splits, chunks_per_split;
+  int n_chunks, n_ctas;
+  long long total_chunks;
+  long long n_slots() const { return total_chunks / n_chunks + n_ctas - 1; }
 };
 
 DecodeSplit decode_split(int B, int Hkv, int Nk, int num_splits) {
   const int n_chunks = (Nk + kTileN - 1) / kTileN;
-  const long long base = (long long)B * Hkv;
-  long long want = num_splits > 0 ? num_splits : (kDecodeTargetCtas + base - 1) / base;
-  want = std::max(1LL, std::min<long long>({want, (long long)n_chunks, (long long)kDecodeMaxSplits}));
-  const int cps = (int)((n_chunks + want - 1) / want);
-  return {(n_chunks + cps - 1) / cps, cps};
+  const long long total = (long long)B * Hkv * n_chunks;
+  const long long want = num_splits > 0 ? (long long)B * Hkv * num_splits : kDecodeSms;
+  return {n_chunks, (int)std::min(want, total), total};
 }
 
 int check_decode(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale) {
@@ -281,10 +283,10 @@ int check_decode(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, floa
   return FA_OK;
 }
 
-size_t decode_workspace(int B, int Hq, int Nq, int d, const DecodeSplit& sp) {
-  const size_t rows = (size_t)B * Hq * Nq;
-  const size_t opart = ((size_t)sp.n_splits * rows * d * sizeof(float) + 255) & ~size_t(255);
-  return opart + (size_t)sp.n_splits * rows * sizeof(float);
+size_t decode_workspace(int B, int Hq, int Hkv, int Nq, int d, const DecodeSplit& sp) {
+  const size_t rows = (size_t)(Hq / Hkv) * Nq;  // query rows of a group
+  const size_t opart = ((size_t)sp.n_slots() * rows * d * sizeof(float) + 255) & ~size_t(255);
+  return opart + (size_t)sp.n_slots() * rows * sizeof(float);
 }
 
 }  // namespace
@@ -294,7 +296,7 @@ extern "C" {
 
 size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {
   if (check_decode(B, Hq, Hkv, Nq, Nk, d, 0, 1.f) != FA_OK) return 0;
-  return decode_workspace(B, Hq, Nq, d, decode_split(B, Hkv, Nk, num_splits));
+  return decode_workspace(B, Hq, Hkv, Nq, d, decode_split(B, Hkv, Nk, num_splits));
 }
 
 int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace, int B, int Hq,
@@ -316,7 +318,8 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.o = o;
   p.lse = lse;
   p.o_part = static_cast<float*>(workspace);
-  const size_t opart = ((size_t)sp.n_splits * rows * d * sizeof(float) + 255) & ~size_t(255);
+  const int g_rows = (Hq / Hkv) * Nq;
+  const size_t opart = ((size_t)sp.n_slots() * g_rows * d * sizeof(float) + 255) & ~size_t(255);
   p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + opart);
   p.status = di->status;
   p.B = B;
@@ -325,8 +328,10 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.Nq = Nq;
   p.Nk = Nk;
   p.causal = causal ? 1 : 0;
-  p.n_splits = sp.n_splits;
-  p.chunks_per_split = sp.chunks_per_split;
+  p.rows = g_rows;
+  p.n_chunks = sp.n_chunks;
+  p.n_ctas = sp.n_ctas;
+  p.total_chunks = sp.total_chunks;
   p.rows_total = rows;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_budget_ns = g_wait_budget_ns.load();

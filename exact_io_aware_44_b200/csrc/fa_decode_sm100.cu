@@ -5,33 +5,42 @@
 // by reading that cache from device memory, which the kernel cannot avoid
 // ("FlashAttention Kernel & Online Softmax" card: the relation to the KV cache
 // and the decode bandwidth bottleneck). So the design goal is to read K and V
-// exactly once at full bandwidth: one CTA handles all query rows of one GQA
-// group (g query heads x Nq queries, at most 32 rows) against one slice of the
-// keys, and enough slices run side by side to fill the GPU.
+// exactly once at full bandwidth. A GQA group (one batch entry and kv head: g
+// query heads x Nq queries, at most 32 rows) is the unit that shares K and V; its
+// keys form n_chunks chunks of 128. All groups' chunks are laid end to end, and
+// CTA i of the persistent grid (one CTA per SM) takes the i-th of n_ctas equal
+// slices of that sequence. A slice may cross group boundaries: each piece of it
+// that lies in one group is a segment, with its own partial output O_s and
+// log-sum-exp LSE_s, stored in slot (group + i) of the workspace. The key ring
+// keeps streaming across segments, so an SM never waits for a new CTA to fill it.
+// decode_merge_kernel combines a group's segments with the online-softmax merge
+// (running max and rescaled denominators, the same update the pages give for key
+// blocks): LSE = log sum_s e^(LSE_s), O = sum_s e^(LSE_s - LSE) O_s.
 //
-// Each split produces an unnormalised-then-normalised partial output O_s and its
-// log-sum-exp LSE_s; decode_merge_kernel combines them with the online-softmax
-// merge (running max and rescaled denominators, the same update the pages give
-// for key blocks): LSE = log sum_s e^(LSE_s), O = sum_s e^(LSE_s - LSE) O_s.
-//
-// decode_split_kernel (192 threads, d = 128):
-//   warp 0      TMA producer: the group's query rows once, then K and V chunks of
-//               128 keys through a 3-stage ring.
-//   warp 1      allocates TMEM (64 or 128 columns); lane 0 issues the MMAs:
+// decode_split_kernel<R> (R = 16 or 32 query rows; 64 + 128 * R / 16 threads; d = 128):
+//   warp 0      TMA producer: each segment's query rows (two buffers, by segment
+//               parity), and K and V chunks of 128 keys through a 3-stage ring.
+//   warp 1      allocates TMEM (4R columns); lane 0 issues the MMAs:
 //                 S^T(c) = K_c Q^T   M = 128 keys, N = R query rows, K = d -> TMEM
 //                 O^T   += V_c^T P^T  M = d = 128, N = R, K = 128 keys      -> TMEM
 //               so keys, and then head-dim columns, sit in TMEM lanes and the few
 //               query rows are the MMA's N (tcgen05 needs M >= 64, N may be 16).
-//   warps 2-5   thread = TMEM lane: key row of S^T, head-dim row of O^T.
+//   warps 2-5   thread = TMEM lane: key row of S^T, head-dim row of O^T; query rows
+//               (TMEM columns) 0-15. For R = 32, warps 6-9 do the same for rows 16-31,
+//               so every softmax thread handles 16 rows and two softmax warps share
+//               each SM sub-partition.
 // The kernel is instantiated for R = 16 and R = 32 query rows (the host takes the
-// smaller that holds the group). Per chunk a thread loads its R scores, and the CTA keeps one reference max per
-// query row, raised only when some score exceeds it by more than 2^8 (the exact
-// column max is then reduced across the 128 threads and O^T and the per-thread
-// partial denominators are rescaled); otherwise P = 2^(S c - m_ref) directly.
-// P^T goes to shared memory as the MMA's B operand (K-major, 128-byte swizzle).
-// The denominators are per-thread partial sums, reduced once at the end.
+// smaller that holds the group). Per chunk a thread loads its 16 scores, and the
+// CTA keeps one reference max per query row for the segment, raised only when
+// some score exceeds it by more than 2^8 (the exact column max is then reduced
+// across the 128 threads and O^T and the per-thread partial denominators are
+// rescaled); otherwise P = 2^(S c - m_ref) directly. P^T goes to shared memory as
+// the MMA's B operand (K-major, 128-byte swizzle). The denominators are per-thread
+// partial sums, reduced at the end of each segment.
 //
-// TMEM columns: S^T buffers [0,R) and [R,2R) (chunk parity), O^T [2R,3R).
+// TMEM columns: S^T buffers [0,R) and [R,2R) (chunk parity), O^T buffers [2R,3R)
+// and [3R,4R) (segment parity), so a segment's output is read while the next
+// segment accumulates.
 #include <math.h>
 
 #include "fa.h"
@@ -41,7 +50,6 @@
 namespace fa {
 namespace {
 
-constexpr int kDecThreads = 192;
 constexpr int kDecChunk = 128;   // keys per chunk (the MMA M)
 constexpr int kDecStages = 3;
 constexpr uint32_t kDecRescaleLog2 = 8;
@@ -50,24 +58,38 @@ constexpr uint32_t kDecRescaleLog2 = 8;
 template <int R>
 struct DecCfg {
   static constexpr int D = 128;
+  static constexpr int kHalves = R / 16;                 // softmax warpgroups, 16 query rows each
+  static constexpr int kThreads = 64 + 128 * kHalves;
   static constexpr int kKV = kDecChunk * D * 2;          // one K or V chunk (32 KB)
   static constexpr int kRegion = kDecChunk * 128;        // 64-column block of a chunk (16 KB)
   static constexpr int kQRegion = R * 128;               // 64-column block of the query tile
   static constexpr int kPRegion = R * 128;               // 64-key block of a P^T tile
-  static constexpr int kOffQ = 0;                        // 2 blocks
-  static constexpr int kOffP = kOffQ + 2 * kQRegion;     // 2 buffers x 2 blocks
+  static constexpr int kOffQ = 0;                        // 2 buffers x 2 blocks
+  static constexpr int kOffP = kOffQ + 4 * kQRegion;     // 2 buffers x 2 blocks
   static constexpr int kOffKV = kOffP + 4 * kPRegion;    // stages of K then V
-  static constexpr int kOffRed = kOffKV + kDecStages * 2 * kKV;   // [3][4][R] floats, then flags [2][4]
+  static constexpr int kOffRed = kOffKV + kDecStages * 2 * kKV;   // [3][4][R] floats, then flags [2][8]
   static constexpr int kOffBar = kOffRed + 3 * 4 * R * 4 + 64;
-  // q_full, kv_full[3], kv_empty[3], s_full[2], p_full[2], pv_done[2], vote[2], red_bar, mma_done
-  static constexpr int kNumBars = 17;
+  // q_full[2], q_empty[2], kv_full[3], kv_empty[3], s_full[2], p_full[2], pv_done[2], vote[2],
+  // red_bar, mma_done
+  static constexpr int kNumBars = 20;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static_assert(kOffKV % 1024 == 0 && kOffP % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  // TMEM: S^T buffers [0, R) and [R, 2R) (chunk parity), O^T [2R, 3R)
   static constexpr int kColS = 0, kColO = 2 * R;
-  static constexpr int kTmemCols = R == 16 ? 64 : 128;
+  static constexpr int kTmemCols = 4 * R;
+};
+
+// Position in a CTA's chunk sequence: group G, chunk of the group cig, segment seg.
+struct ChunkPos {
+  int G, cig, seg;
+  __device__ __forceinline__ void next(int n_chunks) {
+    if (++cig == n_chunks) {
+      cig = 0;
+      ++G;
+      ++seg;
+    }
+  }
 };
 
 __device__ __forceinline__ uint8_t* align1024d(uint8_t* p) {
@@ -99,24 +121,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
-// R-column forms (R = 16 or 32).
-template <int R>
-__device__ __forceinline__ void tmem_ld_r(uint32_t taddr, uint32_t (&r)[R]) {
-  if constexpr (R == 16) {
-    tmem_ld16(taddr, r);
-    tmem_ld_wait16(r);
-  } else {
-    tmem_ld32(taddr, r);
-    tmem_ld_wait(r);
-  }
-}
-template <int R>
-__device__ __forceinline__ void tmem_st_r(uint32_t taddr, const uint32_t (&r)[R]) {
-  if constexpr (R == 16)
-    tmem_st16(taddr, r);
-  else
-    tmem_st32(taddr, r);
-}
 __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
@@ -127,68 +131,68 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, mbar_wait_ns(bar, parity, w, kConsumerPollNs));
 }
 
-// All 128 threads of the softmax warpgroup arrive on `bar` and wait for the phase
-// to complete (a bounded stand-in for a named barrier).
+// Every softmax warp arrives on `bar` once (lane 0, after the warp's own shared-memory
+// accesses are ordered by __syncwarp) and waits for the phase to complete: a bounded
+// stand-in for a named barrier. The barrier counts warps.
 __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, const WaitCtx& w) {
-  mbar_arrive(bar);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
   const bool ok = warp_wait(bar, phase, w);
   phase ^= 1u;
   return ok;
 }
 
 template <int R>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(DecCfg<R>::kThreads, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
   using C = DecCfg<R>;
-  constexpr int kDecRows = R;
+  constexpr int kRows = 16;  // query rows (TMEM columns) per softmax thread
+  constexpr int kSoftmax = 128 * C::kHalves;
   constexpr int S = kDecStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024d(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 4;
-  uint64_t* s_full = bars + 7;
-  uint64_t* p_full = bars + 9;
-  uint64_t* pv_done = bars + 11;
-  uint64_t* vote_bar = bars + 13;
-  uint64_t* red_bar = bars + 15;
-  uint64_t* mma_done = bars + 16;
+  uint64_t* q_empty = bars + 2;
+  uint64_t* kv_full = bars + 4;
+  uint64_t* kv_empty = bars + 7;
+  uint64_t* s_full = bars + 10;
+  uint64_t* p_full = bars + 12;
+  uint64_t* pv_done = bars + 14;
+  uint64_t* vote_bar = bars + 16;
+  uint64_t* red_bar = bars + 18;
+  uint64_t* mma_done = bars + 19;
   // [3][4][R]: column maxima by chunk parity, then the final denominators
   float* red = reinterpret_cast<float*>(smem + C::kOffRed);
-  volatile int* flags = reinterpret_cast<volatile int*>(smem + C::kOffRed + 3 * 4 * R * 4);  // [2][4]
+  volatile int* flags = reinterpret_cast<volatile int*>(smem + C::kOffRed + 3 * 4 * R * 4);  // [2][8]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
-  const int bkv = blockIdx.y;  // b * Hkv + kv head
-  const int b = bkv / p.Hkv;
-  const int kvh = bkv % p.Hkv;
-  const int g = p.Hq / p.Hkv;
-  const int rows = g * p.Nq;                                 // valid query rows (<= R)
-  const int row0 = (b * p.Hq + kvh * g) * p.Nq;              // first global query row
-  const int n_chunks_all = (p.Nk + kDecChunk - 1) / kDecChunk;
-  const int c_begin = min(split * p.chunks_per_split, n_chunks_all);
-  const int c_end = min(c_begin + p.chunks_per_split, n_chunks_all);
-  const int n = c_end - c_begin;                             // chunks of this split
-  const int k_end = min(c_end * kDecChunk, p.Nk);
+  const int nch = p.n_chunks;                     // chunks per group
+  const int rows = p.rows;                        // query rows of a group (<= R)
+  // this CTA's slice [f0, f1) of all groups' chunks laid end to end
+  const long long f0 = (long long)blockIdx.x * p.total_chunks / p.n_ctas;
+  const long long f1 = (long long)(blockIdx.x + 1) * p.total_chunks / p.n_ctas;
+  const int n = (int)(f1 - f0);                   // >= 1: the host launches at most one CTA per chunk
+  const ChunkPos pos0{(int)(f0 / nch), (int)(f0 % nch), 0};
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 1);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], kSoftmax / 32);
+      mbar_init(&pv_done[b], 1);
+      mbar_init(&vote_bar[b], kSoftmax / 32);
+    }
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
-      mbar_init(&pv_done[t], 1);
-      mbar_init(&vote_bar[t], 128);
-    }
-    mbar_init(red_bar, 128);
+    mbar_init(red_bar, kSoftmax / 32);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -205,24 +209,32 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n > 0) {
+    if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, 2 * C::kQRegion);
-      for (int z = 0; z < 2; ++z) tma_load_3d(smem + C::kOffQ + z * C::kQRegion, &tmQ, q_full, z * 64, row0, 0);
       bool ok = true;
-      int issued = 0;
-      for (int c = 0; c < n && ok; ++c) {
+      int issued = 0, q_issued = 0;
+      ChunkPos ps = pos0;
+      for (int c = 0; c < n && ok; ++c, ps.next(nch)) {
+        if (c == 0 || ps.cig == 0) {  // a new segment: its group's query rows
+          const int k = ps.seg;
+          if (!(ok = mbar_wait_spin(&q_empty[k & 1], ((k >> 1) & 1) ^ 1, w))) break;
+          ++q_issued;
+          mbar_arrive_expect_tx(&q_full[k & 1], 2 * C::kQRegion);
+          for (int z = 0; z < 2; ++z)
+            tma_load_3d(smem + C::kOffQ + ((k & 1) * 2 + z) * C::kQRegion, &tmQ, &q_full[k & 1], z * 64,
+                        ps.G * rows, 0);
+        }
         const int s = c % S;
         if (!(ok = mbar_wait_spin(&kv_empty[s], ((c / S) & 1) ^ 1, w))) break;
         ++issued;
         mbar_arrive_expect_tx(&kv_full[s], 2 * C::kKV);
-        const int key0 = (c_begin + c) * kDecChunk;
+        const int key0 = ps.cig * kDecChunk;
         uint8_t* st = smem + C::kOffKV + s * 2 * C::kKV;
         for (int z = 0; z < 2; ++z) {
-          tma_load_3d(st + z * C::kRegion, &tmK, &kv_full[s], z * 64, key0, bkv);
-          tma_load_3d(st + C::kKV + z * C::kRegion, &tmV, &kv_full[s], z * 64, key0, bkv);
+          tma_load_3d(st + z * C::kRegion, &tmK, &kv_full[s], z * 64, key0, ps.G);
+          tma_load_3d(st + C::kKV + z * C::kRegion, &tmV, &kv_full[s], z * 64, key0, ps.G);
         }
       }
       if (!ok) {  // error path: let the loads already issued land before the CTA exits
@@ -230,61 +242,71 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         volatile int zero = 0;
         drain.abort_flag = &zero;
         for (int c = max(0, issued - S); c < issued; ++c) mbar_wait(&kv_full[c % S], (c / S) & 1, drain);
-        mbar_wait(q_full, 0, drain);
+        for (int k = max(0, q_issued - 2); k < q_issued; ++k) mbar_wait(&q_full[k & 1], (k >> 1) & 1, drain);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     const bool leader = lane == 0;
-    constexpr uint32_t kIdS = idesc_bf16_f32(128, kDecRows, false, false);  // S^T = K Q^T
-    constexpr uint32_t kIdO = idesc_bf16_f32(128, kDecRows, true, false);   // O^T = V^T P^T
+    constexpr uint32_t kIdS = idesc_bf16_f32(128, R, false, false);  // S^T = K Q^T
+    constexpr uint32_t kIdO = idesc_bf16_f32(128, R, true, false);   // O^T = V^T P^T
     const uint64_t d_q = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
     const uint64_t d_p = sdesc_sw128(smem_u32(smem + C::kOffP), 16, 1024);
     const uint64_t d_k = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);           // K-major K
     const uint64_t d_v = sdesc_sw128(smem_u32(smem + C::kOffKV + C::kKV), C::kRegion, 1024);  // V^T
-    auto issue_s = [&](int c) {
+    // S^T(c) with the query rows of its segment; the Q buffer is released after the
+    // segment's last S^T
+    auto issue_s = [&](int c, const ChunkPos& ps) -> bool {
+      const int qb = ps.seg & 1;
+      if (c == 0 || ps.cig == 0) {
+        if (!mbar_wait_spin(&q_full[qb], (ps.seg >> 1) & 1, w)) return false;
+      }
+      if (!mbar_wait_spin(&kv_full[c % S], (c / S) & 1, w)) return false;
+      tc_fence_after();
       const uint64_t a0 = desc_advance(d_k, (c % S) * 2 * C::kKV);
+      const uint64_t b0 = desc_advance(d_q, qb * 2 * C::kQRegion);
 #pragma unroll
       for (int k = 0; k < C::D / 16; ++k) {
         const uint32_t ao = (k >> 2) * C::kRegion + (k & 3) * 32;
         const uint32_t bo = (k >> 2) * C::kQRegion + (k & 3) * 32;
         if (leader)
-          mma_bf16_ss(tmem + C::kColS + (c & 1) * R, desc_advance(a0, ao), desc_advance(d_q, bo), kIdS,
+          mma_bf16_ss(tmem + C::kColS + (c & 1) * R, desc_advance(a0, ao), desc_advance(b0, bo), kIdS,
                       k > 0 ? 1u : 0u);
       }
-      if (leader) mma_commit(&s_full[c & 1]);
+      if (leader) {
+        mma_commit(&s_full[c & 1]);
+        if (c == n - 1 || ps.cig == nch - 1) mma_commit(&q_empty[qb]);
+      }
+      return true;
     };
-    auto issue_pv = [&](int c) {
+    // O^T += V^T P^T(c) into the O^T buffer of its segment, overwriting at a segment's first chunk
+    auto issue_pv = [&](int c, const ChunkPos& pp) {
       const uint64_t a0 = desc_advance(d_v, (c % S) * 2 * C::kKV);
       const uint64_t b0 = desc_advance(d_p, (c & 1) * 2 * C::kPRegion);
+      const bool first = c == 0 || pp.cig == 0;
 #pragma unroll
       for (int k = 0; k < kDecChunk / 16; ++k) {
         const uint32_t bo = (k >> 2) * C::kPRegion + (k & 3) * 32;
         if (leader)
-          mma_bf16_ss(tmem + C::kColO, desc_advance(a0, k * 2048), desc_advance(b0, bo), kIdO,
-                      (c > 0 || k > 0) ? 1u : 0u);
+          mma_bf16_ss(tmem + C::kColO + (pp.seg & 1) * R, desc_advance(a0, k * 2048), desc_advance(b0, bo), kIdO,
+                      (!first || k > 0) ? 1u : 0u);
       }
       if (leader) {
         mma_commit(&pv_done[c & 1]);
         mma_commit(&kv_empty[c % S]);
       }
     };
-    bool ok = n == 0 || mbar_wait_spin(q_full, 0, w);
-    tc_fence_after();
-    for (int c = 0; c < 2 && c < n && ok; ++c) {
-      if (!(ok = mbar_wait_spin(&kv_full[c % S], (c / S) & 1, w))) break;
-      tc_fence_after();
-      issue_s(c);
-    }
-    for (int c = 0; c < n && ok; ++c) {
+    bool ok = true;
+    ChunkPos ps = pos0, pp = pos0;  // ps runs two chunks ahead of pp
+    for (int c = 0; c < 2 && c < n && ok; ++c, ps.next(nch)) ok = issue_s(c, ps);
+    for (int c = 0; c < n && ok; ++c, pp.next(nch)) {
       if (!(ok = mbar_wait_spin(&p_full[c & 1], (c >> 1) & 1, w))) break;
       tc_fence_after();
-      issue_pv(c);
+      issue_pv(c, pp);
       // S^T(c + 2) into the buffer whose scores the softmax has read (p_full(c))
       if (c + 2 < n) {
-        if (!(ok = mbar_wait_spin(&kv_full[(c + 2) % S], ((c + 2) / S) & 1, w))) break;
-        tc_fence_after();
-        issue_s(c + 2);
+        if (!(ok = issue_s(c + 2, ps))) break;
+        ps.next(nch);
       }
     }
     if (leader) mma_commit(mma_done);
@@ -295,77 +317,91 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     mbar_wait(mma_done, 0, drain);
   } else {
     // ------------------------------------------------------------ softmax (thread = TMEM lane)
+    // Warpgroup h (warps 2 + 4h .. 5 + 4h) owns query rows [16h, 16h + 16).
     const int quarter = warp & 3;
     const int t = quarter * 32 + lane;
-    const int wq = warp - 2;  // 0..3, index into the reduction arrays
+    const int wq = (warp - 2) & 3;   // 0..3 within the warpgroup, index into the reduction arrays
+    const int h = (warp - 2) >> 2;   // warpgroup
+    const int jr0 = h * kRows;       // first query row of this warpgroup
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float c2 = p.scale_log2;
-    float m_ref[kDecRows], l_part[kDecRows];
-#pragma unroll
-    for (int j = 0; j < kDecRows; ++j) {
-      m_ref[j] = -INFINITY;
-      l_part[j] = 0.f;
-    }
+    float m_ref[kRows], l_part[kRows];
     // Row j is query i = j mod Nq of its head; with the causal mask it sees keys up to
     // Nk - Nq + i. Keys up to all_vis are seen by every valid row.
-    const uint32_t row_mask = rows >= 32 ? 0xffffffffu : ((1u << rows) - 1u);
+    const int my_rows = min(max(rows - jr0, 0), kRows);
+    const uint32_t row_mask = (1u << my_rows) - 1u;
     const int all_vis = p.causal ? p.Nk - p.Nq : p.Nk - 1;
     uint32_t vote_ph[2] = {0, 0}, red_ph = 0;
     bool ok = true;
-    for (int c = 0; c < n && ok; ++c) {
+    ChunkPos pos = pos0;
+    for (int c = 0; c < n && ok; ++c, pos.next(nch)) {
+      const bool seg_first = c == 0 || pos.cig == 0;
+      const bool seg_last = c == n - 1 || pos.cig == nch - 1;
+      const uint32_t o_col = C::kColO + (pos.seg & 1) * R + jr0;
+      if (seg_first) {
+#pragma unroll
+        for (int j = 0; j < kRows; ++j) {
+          m_ref[j] = -INFINITY;
+          l_part[j] = 0.f;
+        }
+      }
       if (!(ok = warp_wait(&s_full[c & 1], (c >> 1) & 1, w))) break;
       tc_fence_after();
-      uint32_t r[R];
-      tmem_ld_r<R>(tmem + lane_off + C::kColS + (c & 1) * R, r);
-      const int key = (c_begin + c) * kDecChunk + t;
-      uint32_t vis = key < k_end ? row_mask : 0u;  // bit j: row j sees this key
-      if (key < k_end && key > all_vis) {           // the causal edge, in the last chunk only
+      uint32_t r[kRows];
+      tmem_ld16(tmem + lane_off + C::kColS + (c & 1) * R + jr0, r);
+      tmem_ld_wait16(r);
+      const int key = pos.cig * kDecChunk + t;
+      uint32_t vis = key < p.Nk ? row_mask : 0u;  // bit j: row jr0 + j sees this key
+      if (key < p.Nk && key > all_vis) {          // the causal edge, in a group's last chunk only
         vis = 0u;
-        for (int j = 0; j < rows; ++j)
-          if (key <= p.Nk - p.Nq + j % p.Nq) vis |= 1u << j;
+        for (int j = 0; j < my_rows; ++j)
+          if (key <= p.Nk - p.Nq + (jr0 + j) % p.Nq) vis |= 1u << j;
       }
-      float x[kDecRows];
+      float x[kRows];
       bool over = false;
 #pragma unroll
-      for (int j = 0; j < kDecRows; ++j) {
+      for (int j = 0; j < kRows; ++j) {
         x[j] = (vis >> j) & 1u ? __uint_as_float(r[j]) * c2 : -INFINITY;
         over |= x[j] > m_ref[j] + (float)kDecRescaleLog2;
       }
       // does any thread need a higher reference max for some row?
       const int wv = __any_sync(0xffffffffu, over);
-      if (lane == 0) flags[(c & 1) * 4 + wq] = wv;
+      if (lane == 0) flags[(c & 1) * 8 + (warp - 2)] = wv;
       if (!(ok = group_sync(&vote_bar[c & 1], vote_ph[c & 1], w))) break;
-      const bool rescale = flags[(c & 1) * 4 + 0] | flags[(c & 1) * 4 + 1] | flags[(c & 1) * 4 + 2] |
-                           flags[(c & 1) * 4 + 3];
-      if (rescale) {
-        // exact column max of this chunk over the 128 threads
+      int any = 0;
+#pragma unroll
+      for (int f = 0; f < 4 * C::kHalves; ++f) any |= flags[(c & 1) * 8 + f];
+      if (any) {
+        // exact column max of this chunk over the 128 threads of the warpgroup
         float* rd = red + (c & 1) * 4 * R;
 #pragma unroll
-        for (int j = 0; j < kDecRows; ++j) {
+        for (int j = 0; j < kRows; ++j) {
           float v = x[j];
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == 0) rd[wq * R + j] = v;
+          if (lane == 0) rd[wq * R + jr0 + j] = v;
         }
         if (!(ok = group_sync(red_bar, red_ph, w))) break;
-        float alpha[kDecRows];
+        float alpha[kRows];
 #pragma unroll
-        for (int j = 0; j < kDecRows; ++j) {
-          const float cm = fmaxf(fmaxf(rd[j], rd[R + j]), fmaxf(rd[2 * R + j], rd[3 * R + j]));
+        for (int j = 0; j < kRows; ++j) {
+          const int q = jr0 + j;
+          const float cm = fmaxf(fmaxf(rd[q], rd[R + q]), fmaxf(rd[2 * R + q], rd[3 * R + q]));
           const float m_new = fmaxf(m_ref[j], cm);
           alpha[j] = (m_new == -INFINITY || m_ref[j] == m_new) ? 1.f : ex2(m_ref[j] - m_new);
           m_ref[j] = m_new;
           l_part[j] *= alpha[j];
         }
-        // O^T (thread = head-dim row) once every earlier P V is complete
-        if (c > 0) {
+        // the segment's O^T (thread = head-dim row) once every earlier P V of it is complete
+        if (!seg_first) {
           if (!(ok = warp_wait(&pv_done[(c - 1) & 1], ((c - 1) >> 1) & 1, w))) break;
           tc_fence_after();
-          uint32_t o[R];
-          tmem_ld_r<R>(tmem + lane_off + C::kColO, o);
+          uint32_t o[kRows];
+          tmem_ld16(tmem + lane_off + o_col, o);
+          tmem_ld_wait16(o);
 #pragma unroll
-          for (int j = 0; j < kDecRows; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha[j]);
-          tmem_st_r<R>(tmem + lane_off + C::kColO, o);
+          for (int j = 0; j < kRows; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha[j]);
+          tmem_st16(tmem + lane_off + o_col, o);
           tmem_st_wait();
         }
       }
@@ -376,50 +412,46 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const uint32_t pbuf = smem_u32(smem + C::kOffP + (c & 1) * 2 * C::kPRegion) + (t >> 6) * C::kPRegion;
       const uint32_t kb = (uint32_t)(t & 63) * 2;  // byte offset of this key within a 128-byte row
 #pragma unroll
-      for (int j = 0; j < kDecRows; ++j) {
+      for (int j = 0; j < kRows; ++j) {
         const float e = x[j] == -INFINITY ? 0.f : ex2(x[j] - m_ref[j]);
         l_part[j] += e;
         const uint16_t hb = (uint16_t)(pack_bf16x2(e, 0.f) & 0xFFFFu);
-        st_shared_u16(pbuf + sw128_offset(j, kb >> 4) + (kb & 15), hb);
+        st_shared_u16(pbuf + sw128_offset(jr0 + j, kb >> 4) + (kb & 15), hb);
       }
-      fence_async_smem();
+      fence_async_smem();  // every thread's P^T stores, visible to the MMA (async proxy)
       tc_fence_before();
-      mbar_arrive(&p_full[c & 1]);
-    }
-    // epilogue: denominators reduced over the 128 threads, O^T / l -> partial outputs
-    if (ok && n > 0) {
-      float* rd = red + 2 * 4 * R;  // its own slot: a slower thread may still read the last maxima
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[c & 1]);
+      if (seg_last) {
+        // end of a segment: denominators reduced over the 128 threads, O^T / l -> its slot
+        float* rd = red + 2 * 4 * R;  // its own slot: a slower thread may still read the last maxima
 #pragma unroll
-      for (int j = 0; j < kDecRows; ++j) {
-        float v = l_part[j];
+        for (int j = 0; j < kRows; ++j) {
+          float v = l_part[j];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) rd[wq * R + j] = v;
-      }
-      ok = group_sync(red_bar, red_ph, w);
-      if (ok) ok = warp_wait(mma_done, 0, w);
-      if (ok) {
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0) rd[wq * R + jr0 + j] = v;
+        }
+        if (!(ok = group_sync(red_bar, red_ph, w))) break;
+        if (!(ok = warp_wait(&pv_done[c & 1], (c >> 1) & 1, w))) break;
         tc_fence_after();
-        uint32_t o[R];
-        tmem_ld_r<R>(tmem + lane_off + C::kColO, o);
-        float* opart = p.o_part + (size_t)split * p.rows_total * C::D;
+        uint32_t o[kRows];
+        tmem_ld16(tmem + lane_off + o_col, o);
+        tmem_ld_wait16(o);
+        const size_t slot_row = (size_t)(pos.G + (int)blockIdx.x) * rows;
 #pragma unroll
-        for (int j = 0; j < kDecRows; ++j) {
-          if (j < rows) {
-            const float l = rd[j] + rd[R + j] + rd[2 * R + j] + rd[3 * R + j];
+        for (int j = 0; j < kRows; ++j) {
+          if (j < my_rows) {
+            const int q = jr0 + j;
+            const float l = rd[q] + rd[R + q] + rd[2 * R + q] + rd[3 * R + q];
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            opart[(size_t)(row0 + j) * C::D + t] = __uint_as_float(o[j]) * inv;
+            p.o_part[(slot_row + q) * C::D + t] = __uint_as_float(o[j]) * inv;
             if (t == 0)
-              p.lse_part[(size_t)split * p.rows_total + row0 + j] =
-                  l > 0.f ? (m_ref[j] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+              p.lse_part[slot_row + q] = l > 0.f ? (m_ref[j] + log2f(l)) * 0.6931471805599453f : -INFINITY;
           }
         }
+        tc_fence_before();  // the O^T reads, before a later segment's P V overwrites the buffer
       }
-    }
-    if (n == 0 && t < rows) {  // an empty split contributes nothing
-      p.lse_part[(size_t)split * p.rows_total + row0 + t] = -INFINITY;
-      float* opart = p.o_part + ((size_t)split * p.rows_total + row0 + t) * C::D;
-      for (int dd = 0; dd < C::D; ++dd) opart[dd] = 0.f;
     }
   }
 
@@ -431,19 +463,31 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 }
 
-// One block per query row, one thread per head-dim column: the split partials
-// combined with the online-softmax merge, O in bf16 and LSE.
+// The CTA whose slice of the chunk sequence holds chunk x: the largest i with
+// floor(i * total / n_ctas) <= x.
+__device__ __forceinline__ int decode_cta_of(long long x, const DecodeParams& p) {
+  return (int)(((x + 1) * p.n_ctas - 1) / p.total_chunks);
+}
+
+// One block per query row, one thread per head-dim column: the row's group's
+// segments (slots group + i for the CTAs i that covered it) combined with the
+// online-softmax merge, O in bf16 and LSE.
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p) {
   const long long row = blockIdx.x;
   const int t = threadIdx.x;
+  const int G = (int)(row / p.rows);
+  const int q = (int)(row % p.rows);
+  const int i0 = decode_cta_of((long long)G * p.n_chunks, p);
+  const int i1 = decode_cta_of((long long)(G + 1) * p.n_chunks - 1, p);
   float m = -INFINITY;
-  for (int s = 0; s < p.n_splits; ++s) m = fmaxf(m, p.lse_part[(size_t)s * p.rows_total + row]);
+  for (int i = i0; i <= i1; ++i) m = fmaxf(m, p.lse_part[(size_t)(G + i) * p.rows + q]);
   float wsum = 0.f, acc = 0.f;
-  for (int s = 0; s < p.n_splits; ++s) {
-    const float ls = p.lse_part[(size_t)s * p.rows_total + row];
+  for (int i = i0; i <= i1; ++i) {
+    const size_t slot_row = (size_t)(G + i) * p.rows + q;
+    const float ls = p.lse_part[slot_row];
     const float wgt = ls == -INFINITY ? 0.f : __expf(ls - m);
     wsum += wgt;
-    acc += wgt * p.o_part[((size_t)s * p.rows_total + row) * 128 + t];
+    acc += wgt * p.o_part[slot_row * 128 + t];
   }
   const float o = wsum > 0.f ? acc / wsum : 0.f;
   static_cast<__nv_bfloat16*>(p.o)[row * 128 + t] = __float2bfloat16_rn(o);
@@ -463,8 +507,7 @@ cudaError_t launch_decode_r(const CUtensorMap& tq, const CUtensorMap& tk, const 
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  dim3 grid((unsigned)p.n_splits, (unsigned)(p.B * p.Hkv));
-  decode_split_kernel<R><<<grid, kDecThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
+  decode_split_kernel<R><<<(unsigned)p.n_ctas, C::kThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<(unsigned)p.rows_total, 128, 0, s>>>(p);
@@ -475,8 +518,8 @@ int decode_rows_per_cta(int rows) { return rows <= 16 ? 16 : 32; }
 
 cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           cudaStream_t s) {
-  const int rows = (p.Hq / p.Hkv) * p.Nq;
-  return decode_rows_per_cta(rows) == 16 ? launch_decode_r<16>(tq, tk, tv, p, s) : launch_decode_r<32>(tq, tk, tv, p, s);
+  return decode_rows_per_cta(p.rows) == 16 ? launch_decode_r<16>(tq, tk, tv, p, s)
+                                           : launch_decode_r<32>(tq, tk, tv, p, s);
 }
 
 }  // namespace fa

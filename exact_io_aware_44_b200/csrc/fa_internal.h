@@ -49,12 +49,15 @@ struct BwdParams {
 struct DecodeParams {
   void* o;            // bf16 [B, Hq, Nq, d]
   float* lse;         // [B, Hq, Nq]
-  float* o_part;      // workspace: per split, normalised partial O [n_splits, B * Hq * Nq, d]
-  float* lse_part;    // workspace: per split, partial LSE (natural log) [n_splits, B * Hq * Nq]
+  float* o_part;      // workspace: per segment slot, normalised partial O [n_slots, rows, d]
+  float* lse_part;    // workspace: per segment slot, partial LSE (natural log) [n_slots, rows]
   int* status;
   int B, Hq, Hkv, Nq, Nk;
   int causal;
-  int n_splits, chunks_per_split;  // key splits and 128-key chunks per split
+  int rows;                        // query rows of a GQA group: (Hq / Hkv) * Nq
+  int n_chunks;                    // 128-key chunks per group
+  int n_ctas;                      // split-kernel CTAs (equal slices of all groups' chunks)
+  long long total_chunks;          // B * Hkv * n_chunks
   long long rows_total;            // B * Hq * Nq
   float scale_log2;
   uint64_t wait_budget_ns;

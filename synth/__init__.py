@@ -255,6 +255,8 @@ class DecodeWorkload:
 DECODE_WORKLOADS = {
     # one decode step of a GQA model (32 query heads, 8 kv heads) over a 32K-token cache
     "dec": DecodeWorkload("dec", 16, 32, 8, 1, 32768, 128, True, 1010),
+    # speculative / multi-token decode: 4 new tokens per sequence, GQA group 8 (32 query rows a CTA)
+    "dec4": DecodeWorkload("dec4", 16, 32, 4, 4, 32768, 128, True, 1011),
 }
 
 

@@ -99,19 +99,27 @@ def test_decode_rejects_bad_arguments_on_host():
     assert _dec(ws=0) == -1
 
 
+def _decode_slots(B, Hq, Hkv, Nq, Nk, splits):
+    """The work split restated: all groups' 128-key chunks end to end, cut into
+    n_ctas equal slices (one per SM of a 148-SM part, or B * Hkv * num_splits;
+    never more than the chunks); one workspace slot per (group, CTA) pair that
+    can meet, i.e. groups + n_ctas - 1."""
+    n_chunks = -(-Nk // 128)
+    total = B * Hkv * n_chunks
+    n_ctas = min(B * Hkv * splits if splits > 0 else 148, total)
+    return B * Hkv + n_ctas - 1
+
+
 def test_decode_workspace_and_split_rule():
-    """Per split: fp32 partial O (256-byte padded) and fp32 partial LSE per query row."""
-    B, Hq, Hkv, Nq, d = 4, 32, 8, 1, 128
-    for Nk, splits in ((128, 1), (4096, 4), (4096, 7), (100000, 0)):
-        ws = fa.decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, splits)
-        n_chunks = -(-Nk // 128)
-        want = splits if splits > 0 else -(-296 // (B * Hkv))
-        want = max(1, min(want, n_chunks, 256))
-        cps = -(-n_chunks // want)
-        ns = -(-n_chunks // cps)
-        rows = B * Hq * Nq
-        opart = (ns * rows * d * 4 + 255) // 256 * 256
-        assert ws == opart + ns * rows * 4, (Nk, splits, ws)
+    """Per slot: fp32 partial O (256-byte padded) and fp32 partial LSE per query row of a group."""
+    d = 128
+    for (B, Hq, Hkv, Nq) in ((4, 32, 8, 1), (16, 32, 8, 1), (16, 32, 4, 4), (1, 8, 1, 3), (64, 16, 8, 1)):
+        for Nk, splits in ((128, 1), (4096, 4), (4096, 7), (100000, 0), (32768, 0), (777, 0), (1, 0), (200, 0)):
+            ws = fa.decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, splits)
+            slots = _decode_slots(B, Hq, Hkv, Nq, Nk, splits)
+            rows = Hq // Hkv * Nq
+            opart = (slots * rows * d * 4 + 255) // 256 * 256
+            assert ws == opart + slots * rows * 4, (B, Hq, Hkv, Nq, Nk, splits, ws)
     assert fa.decode_workspace_bytes(1, 8, 1, 1, 1000, 64, 0) == 0
 
 

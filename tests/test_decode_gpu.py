@@ -49,6 +49,10 @@ SHAPES = [
     (1, 32, 1, 1, 513),     # a 32-head group
     (1, 2, 1, 16, 640),     # 16 new tokens per head, 32 rows, the causal edge spans 16 keys
     (1, 1, 1, 17, 17),      # square, 17 rows
+    (3, 8, 2, 1, 7000),     # 330 chunks over 148 CTAs: slices cross group boundaries
+    (1, 32, 4, 4, 9000),    # the same with 32 rows
+    (64, 16, 8, 1, 200),    # 1024 chunks of short caches: about 4 segments per CTA
+    (32, 32, 4, 3, 300),    # 24 rows, 3 chunks a group, segments across groups
 ]
 
 
@@ -109,11 +113,13 @@ def test_decode_repeatable_and_bounded_writes(cuda_device):
     assert torch.equal(o_buf[:n_o].view_as(q), o2) and torch.equal(l_buf[:16].view(2, 8, 1), l2)
 
 
-def test_decode_full_size_workload(cuda_device):
-    """The benchmark's decode step (B=16 Hq=32 Hkv=8, one query against 32768
-    cached keys), in the launch configuration the benchmark times (automatic
-    splits); every output computed, sampled heads checked against the oracle."""
-    w = synth.DECODE_WORKLOADS["dec"]
+@pytest.mark.parametrize("name", ["dec", "dec4"])
+def test_decode_full_size_workload(cuda_device, name):
+    """The benchmark's decode steps (B=16 Hq=32 against 32768 cached keys: Hkv=8 with
+    one new query, Hkv=4 with four), in the launch configuration the benchmark
+    times (automatic splits); every output computed, sampled heads checked
+    against the oracle."""
+    w = synth.DECODE_WORKLOADS[name]
     q, k, v, o, lse = run_decode(w, cuda_device)
     assert np.isfinite(o).all() and np.isfinite(lse).all()
     for (b, h) in ((0, 0), (3, 9), (7, 31), (15, 16)):
