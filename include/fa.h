@@ -111,9 +111,12 @@ int fa_fwd_e5m2(const void* q, const void* k, const void* v, float descale_q, fl
 /*
  * fa_decode_workspace_bytes -- device scratch that fa_decode needs.
  *
- * Per key split, a float32 partial output [B*Hq*Nq, d] and a float32 partial
- * LSE [B*Hq*Nq]. num_splits <= 0 means the split count fa_decode chooses itself
- * (a fixed rule of the sizes, so no device is needed here). Returns 0 for sizes
+ * The split kernel cuts all (batch, kv head) groups' 128-key chunks, laid end to
+ * end, into n_ctas equal slices; each piece of a slice inside one group has a
+ * slot holding a float32 partial output [rows, d] and partial LSE [rows], with
+ * rows = (Hq / Hkv) * Nq, and there are B*Hkv + n_ctas - 1 slots. n_ctas is 148
+ * for num_splits <= 0 (a fixed rule of the sizes, so no device is needed here),
+ * else B*Hkv*num_splits, and never more than the chunks. Returns 0 for sizes
  * fa_decode rejects.
  */
 size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits);
@@ -134,8 +137,9 @@ size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, 
  *   o [B,Hq,Nq,d] bf16, lse [B,Hq,Nq] float32   outputs, as in fa_fwd
  *   workspace   at least fa_decode_workspace_bytes(..., num_splits) bytes of
  *               device memory, 256-byte aligned, contents on entry irrelevant
- *   num_splits  key splits (<= 0: chosen from the sizes; capped by the number of
- *               128-key chunks)
+ *   num_splits  work split: <= 0 gives one CTA per SM of a 148-SM part; > 0 gives
+ *               B*Hkv*num_splits CTAs (about num_splits key splits per group); never
+ *               more CTAs than 128-key chunks
  *   d must be 128 and (Hq / Hkv) * Nq at most 32 (one CTA serves a whole GQA
  *   group's query rows), else FA_ERR_UNSUPPORTED; causal with Nq > Nk is
  *   FA_ERR_INVALID_ARG. Arithmetic: bf16 operands, fp32 accumulation; P is
