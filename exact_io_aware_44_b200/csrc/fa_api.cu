@@ -107,6 +107,21 @@ int make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box_
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
 }
 
+// Consecutive heads that the kernels schedule together (the causal work order runs
+// longest-first across them): `per_unit` heads share one unit (a kv head) whose
+// operands are re-read, `reuse_bytes` of them. As many units as keep those within
+// 48 MB, well inside the 126 MB L2, and a divisor of the unit count, so that no
+// short last group ends the launch with long blocks.
+int head_group(double reuse_bytes, int per_unit, int total) {
+  const double budget = 48.0 * 1024 * 1024;
+  const int units = total / per_unit;
+  const long long max_units = std::max(1LL, (long long)(budget / std::max(reuse_bytes, 1.0)));
+  int best = 1;
+  for (int u = 1; u <= units && u <= max_units; ++u)
+    if (units % u == 0) best = u;
+  return best * per_unit;
+}
+
 }  // namespace
 }  // namespace fa
 
@@ -161,6 +176,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.causal = causal ? 1 : 0;
   const int rows_per_cta = fwd_tiles_per_cta(d) * kTileM;
   p.n_qblk = (N + rows_per_cta - 1) / rows_per_cta;
+  p.head_group = head_group(2.0 * N * d * 2, Hq / Hkv, B * Hq);  // K and V of a kv head
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_scale = 1.f;
   p.wait_budget_ns = g_wait_budget_ns.load();
@@ -198,6 +214,7 @@ static int fwd_f8(bool e5m2, const void* q, const void* k, const void* v, float 
   p.N = N;
   p.causal = causal ? 1 : 0;
   p.n_qblk = (N + 2 * kTileM - 1) / (2 * kTileM);
+  p.head_group = head_group(2.0 * N * d, Hq / Hkv, B * Hq);  // K and V of a kv head, one byte each
   p.scale_log2 = c;
   p.o_scale = descale_v;
   p.wait_budget_ns = g_wait_budget_ns.load();
@@ -408,6 +425,8 @@ int run_bwd(int phases, const void* q, const void* k, const void* v, const void*
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
+  // per kv head, for its Hq / Hkv query heads: Q and dO (bf16), the fp32 dQ accumulator, LSE and D
+  p.head_group = head_group((double)(Hq / Hkv) * N * (8.0 * d + 8), 1, B * Hkv);
   p.wait_budget_ns = g_wait_budget_ns.load();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (pre && launch_bwd_preprocess(p, s) != cudaSuccess) return FA_ERR_LAUNCH;

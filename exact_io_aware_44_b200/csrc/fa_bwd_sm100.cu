@@ -199,11 +199,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: (batch, kv head, key tile), key tile 0 first (it sees the most
-  // query tiles under the causal mask).
+  // Work unit: (batch, kv head, key tile). (batch, kv head) pairs in groups of
+  // p.head_group, whose Q, dO and dQ accumulators fit in L2 together; within a group
+  // key tile 0 of every pair first (it sees the most query tiles under the causal mask).
   const int n_kt = (p.N + kTileN - 1) / kTileN;
-  const int kt = blockIdx.x % n_kt;
-  const int bkv = blockIdx.x / n_kt;
+  const int grp0 = (int)(blockIdx.x / (unsigned)(p.head_group * n_kt)) * p.head_group;
+  const int gsz = min(p.head_group, p.B * p.Hkv - grp0);
+  const int r = (int)blockIdx.x - grp0 * n_kt;
+  const int bkv = grp0 + r % gsz;
+  const int kt = r / gsz;
   const int b = bkv / p.Hkv;
   const int kvh = bkv % p.Hkv;
   const int g = p.Hq / p.Hkv;
@@ -652,10 +656,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: (batch, kv head, key tile), key tile 0 first.
+  // Work unit: (batch, kv head, key tile). (batch, kv head) pairs in groups of
+  // p.head_group, whose Q, dO and dQ accumulators fit in L2 together; within a group
+  // key tile 0 of every pair first (it sees the most query tiles under the causal mask).
   const int n_kt = (p.N + kTileN - 1) / kTileN;
-  const int kt = blockIdx.x % n_kt;
-  const int bkv = blockIdx.x / n_kt;
+  const int grp0 = (int)(blockIdx.x / (unsigned)(p.head_group * n_kt)) * p.head_group;
+  const int gsz = min(p.head_group, p.B * p.Hkv - grp0);
+  const int r = (int)blockIdx.x - grp0 * n_kt;
+  const int bkv = grp0 + r % gsz;
+  const int kt = r / gsz;
   const int b = bkv / p.Hkv;
   const int kvh = bkv % p.Hkv;
   const int g = p.Hq / p.Hkv;

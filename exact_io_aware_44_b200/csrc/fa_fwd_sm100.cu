@@ -139,10 +139,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: head-major so that concurrently running CTAs share K/V in L2,
-  // and within a head the longest (last) query blocks first.
-  const int bh = blockIdx.x / p.n_qblk;
-  const int qb = p.n_qblk - 1 - (blockIdx.x % p.n_qblk);
+  // Work unit: heads in groups of p.head_group, whose K/V fit in L2 together, so that
+  // concurrently running CTAs share them; within a group the longest (last) query
+  // blocks of all its heads first, so that the causal tail ends on short blocks.
+  const int grp0 = (int)(blockIdx.x / (unsigned)(p.head_group * p.n_qblk)) * p.head_group;
+  const int gsz = min(p.head_group, p.B * p.Hq - grp0);
+  const int r = (int)blockIdx.x - grp0 * p.n_qblk;
+  const int bh = grp0 + r % gsz;
+  const int qb = p.n_qblk - 1 - r / gsz;
   const int b = bh / p.Hq;
   const int h = bh % p.Hq;
   const int kv_head = b * p.Hkv + h / (p.Hq / p.Hkv);

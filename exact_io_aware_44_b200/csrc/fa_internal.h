@@ -18,6 +18,7 @@ struct FwdParams {
   int B, Hq, Hkv, N;
   int causal;
   int n_qblk;         // query blocks of 2 tiles (256 rows) per head
+  int head_group;     // consecutive (batch, head) pairs scheduled together (a multiple of Hq / Hkv)
   float scale_log2;   // scale * log2(e) (times the Q and K descales for E4M3 inputs)
   float o_scale;      // multiplies O at the end (the V descale for E4M3 inputs, else 1)
   uint64_t wait_budget_ns;
@@ -43,6 +44,7 @@ struct BwdParams {
   int causal;
   float scale;
   float scale_log2;
+  int head_group;    // consecutive (batch, kv head) pairs scheduled together
   uint64_t wait_budget_ns;
 };
 
