@@ -49,8 +49,8 @@ NCU_TRAFFIC = {
     # profiles/bwd_main_d128_B2H32N8192_causal.md
     ("bwd_main", "c3"): {"bytes_per_launch": 810462464 + 489935104, "csrc_sha": "ed7fc08fb60db3a8"},
     # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md
-    ("decode_split", "dec"): {"bytes_per_launch": 2148443904 + 3871232, "csrc_sha": "c1652c60e81fafd1"},
-    ("decode_split", "dec4"): {"bytes_per_launch": 1074819072 + 5263104, "csrc_sha": "c1652c60e81fafd1"},
+    ("decode_split", "dec"): {"bytes_per_launch": 2148211200 + 3646464, "csrc_sha": "fee321784a151a1f"},
+    ("decode_split", "dec4"): {"bytes_per_launch": 1074812160 + 4330240, "csrc_sha": "fee321784a151a1f"},
 }
 
 

@@ -469,29 +469,46 @@ __device__ __forceinline__ int decode_cta_of(long long x, const DecodeParams& p)
   return (int)(((x + 1) * p.n_ctas - 1) / p.total_chunks);
 }
 
-// One block per query row, one thread per head-dim column: the row's group's
-// segments (slots group + i for the CTAs i that covered it) combined with the
-// online-softmax merge, O in bf16 and LSE.
-__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p) {
-  const long long row = blockIdx.x;
-  const int t = threadIdx.x;
+// One warp per query row, four head-dim columns per lane: the row's group's
+// segments (slots group + i for the CTAs i that covered it) combined in one pass
+// with the online-softmax merge (running max, rescaled weight sum and output),
+// then O in bf16 and LSE.
+constexpr int kMergeRowsPerBlock = 8;
+
+__global__ void __launch_bounds__(32 * kMergeRowsPerBlock) decode_merge_kernel(const DecodeParams p) {
+  const long long row = (long long)blockIdx.x * kMergeRowsPerBlock + (threadIdx.x >> 5);
+  if (row >= p.rows_total) return;
+  const int lane = threadIdx.x & 31;
   const int G = (int)(row / p.rows);
   const int q = (int)(row % p.rows);
   const int i0 = decode_cta_of((long long)G * p.n_chunks, p);
   const int i1 = decode_cta_of((long long)(G + 1) * p.n_chunks - 1, p);
-  float m = -INFINITY;
-  for (int i = i0; i <= i1; ++i) m = fmaxf(m, p.lse_part[(size_t)(G + i) * p.rows + q]);
-  float wsum = 0.f, acc = 0.f;
+  float m = -INFINITY, wsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
   for (int i = i0; i <= i1; ++i) {
     const size_t slot_row = (size_t)(G + i) * p.rows + q;
     const float ls = p.lse_part[slot_row];
-    const float wgt = ls == -INFINITY ? 0.f : __expf(ls - m);
-    wsum += wgt;
-    acc += wgt * p.o_part[slot_row * 128 + t];
+    const float4 o4 = reinterpret_cast<const float4*>(p.o_part + slot_row * 128)[lane];
+    if (ls == -INFINITY) continue;  // no visible key in this segment
+    const float m_new = fmaxf(m, ls);
+    const float a = __expf(m - m_new);  // 0 while m is still -inf
+    const float wgt = __expf(ls - m_new);
+    wsum = wsum * a + wgt;
+    acc.x = acc.x * a + wgt * o4.x;
+    acc.y = acc.y * a + wgt * o4.y;
+    acc.z = acc.z * a + wgt * o4.z;
+    acc.w = acc.w * a + wgt * o4.w;
+    m = m_new;
   }
-  const float o = wsum > 0.f ? acc / wsum : 0.f;
-  static_cast<__nv_bfloat16*>(p.o)[row * 128 + t] = __float2bfloat16_rn(o);
-  if (t == 0) p.lse[row] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  uint2 packed;
+  packed.x = *reinterpret_cast<uint32_t*>(&lo);
+  packed.y = *reinterpret_cast<uint32_t*>(&hi);
+  reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.o) + row * 128)[lane] = packed;
+  if (lane == 0) p.lse[row] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
 }
 
 }  // namespace
@@ -510,7 +527,8 @@ cudaError_t launch_decode_r(const CUtensorMap& tq, const CUtensorMap& tk, const 
   decode_split_kernel<R><<<(unsigned)p.n_ctas, C::kThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_merge_kernel<<<(unsigned)p.rows_total, 128, 0, s>>>(p);
+  decode_merge_kernel<<<(unsigned)((p.rows_total + kMergeRowsPerBlock - 1) / kMergeRowsPerBlock),
+                        32 * kMergeRowsPerBlock, 0, s>>>(p);
   return cudaGetLastError();
 }
 
