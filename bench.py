@@ -49,8 +49,8 @@ NCU_TRAFFIC = {
     # profiles/bwd_main_d128_B2H32N8192_causal.md
     ("bwd_main", "c3"): {"bytes_per_launch": 810462464 + 489935104, "csrc_sha": "ed7fc08fb60db3a8"},
     # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md
-    ("decode_split", "dec"): {"bytes_per_launch": 2148211200 + 3646464, "csrc_sha": "fee321784a151a1f"},
-    ("decode_split", "dec4"): {"bytes_per_launch": 1074812160 + 4330240, "csrc_sha": "fee321784a151a1f"},
+    ("decode_split", "dec"): {"bytes_per_launch": 2148211200 + 3646464, "csrc_sha": "23e740588e569a93"},
+    ("decode_split", "dec4"): {"bytes_per_launch": 1074812160 + 4330240, "csrc_sha": "23e740588e569a93"},
 }
 
 
@@ -61,7 +61,7 @@ KERNEL_SOURCES = {
     "bwd_main": ("fa_bwd_sm100.cu", [("__device__ __forceinline__ void red_add_v4", "// ----"),
                                      ("struct Bwd128Cfg {", "int sm_count() {")]),
     "fwd": ("fa_fwd_sm100.cu", [("", None)]),
-    "decode_split": ("fa_decode_sm100.cu", [("", None)]),
+    "decode_split": ("fa_decode_sm100.cu", [("template <int R>\nstruct DecCfg {", "template <int R>\ncudaError_t launch_decode_r(")]),
 }
 
 

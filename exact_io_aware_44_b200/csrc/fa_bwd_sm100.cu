@@ -1063,15 +1063,15 @@ cudaError_t launch_main_d(const CUtensorMap& tq, const CUtensorMap& tk, const CU
   const long long grid = (long long)p.B * p.Hkv * ((p.N + kTileN - 1) / kTileN);
   if constexpr (D == 128) {
     using C = Bwd128Cfg;
-    cudaError_t e =
-        cudaFuncSetAttribute(bwd_main_d128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    static std::atomic<uint64_t> configured{0};
+    cudaError_t e = ensure_smem_limit(bwd_main_d128_kernel, C::kSmemBytes, configured);
     if (e != cudaSuccess) return e;
     bwd_main_d128_kernel<<<(unsigned)grid, kBwdThreads, C::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
   } else {
     using C = BwdCfg<D>;
     static_assert(C::kSmemBytes <= 232448, "shared memory budget");
-    cudaError_t e =
-        cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    static std::atomic<uint64_t> configured{0};
+    cudaError_t e = ensure_smem_limit(bwd_main_kernel<D>, C::kSmemBytes, configured);
     if (e != cudaSuccess) return e;
     bwd_main_kernel<D><<<(unsigned)grid, kBwdThreads, C::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
   }

@@ -517,15 +517,11 @@ template <int R>
 cudaError_t launch_decode_r(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const DecodeParams& p, cudaStream_t s) {
   using C = DecCfg<R>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = ensure_smem_limit(decode_split_kernel<R>, C::kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
   decode_split_kernel<R><<<(unsigned)p.n_ctas, C::kThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<(unsigned)((p.rows_total + kMergeRowsPerBlock - 1) / kMergeRowsPerBlock),
                         32 * kMergeRowsPerBlock, 0, s>>>(p);

@@ -487,13 +487,9 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          cudaStream_t stream) {
   using C = FwdCfg<D, KIND != kKindBf16>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = ensure_smem_limit(fwd_kernel<D, KIND>, C::kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
   const long long grid = (long long)p.B * p.Hq * p.n_qblk;
   fwd_kernel<D, KIND><<<(unsigned)grid, kFwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace fa {
 
 constexpr int kTileM = 128;  // query rows per tile (TMEM lanes)
@@ -88,5 +90,21 @@ cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const CUtensorMap& tdo, const BwdParams& p, cudaStream_t s);
 cudaError_t launch_bwd_convert(const BwdParams& p, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* status, uint64_t budget_ns, cudaStream_t s);
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current device,
+// once per device (the attribute is per device; `done` holds one bit per device
+// ordinal below 64, larger ordinals set it on every call). Thread-safe: a race
+// only repeats the idempotent call.
+template <typename Kernel>
+cudaError_t ensure_smem_limit(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 }  // namespace fa
