@@ -115,11 +115,12 @@ int make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box_
 int head_group(double reuse_bytes, int per_unit, int total) {
   const double budget = 48.0 * 1024 * 1024;
   const int units = total / per_unit;
-  const long long max_units = std::max(1LL, (long long)(budget / std::max(reuse_bytes, 1.0)));
-  int best = 1;
-  for (int u = 1; u <= units && u <= max_units; ++u)
-    if (units % u == 0) best = u;
-  return best * per_unit;
+  // groups of more than 1024 units schedule no better and would only lengthen the search
+  const int max_units = (int)std::min(1024.0, std::max(1.0, budget / std::max(reuse_bytes, 1.0)));
+  if (units <= max_units) return total;
+  for (int u = max_units; u > 1; --u)
+    if (units % u == 0) return u * per_unit;
+  return per_unit;
 }
 
 }  // namespace
