@@ -310,6 +310,15 @@ def pin_decode(dec):
                                                     causal, scale)
                 np.testing.assert_allclose(o[0, h], np.array(ob), rtol=1e-12, atol=1e-12)
                 np.testing.assert_allclose(lse[0, h], np.array(lb), rtol=1e-12, atol=1e-12)
+    # a whole 32-row group (8 query heads on one kv head x 4 new tokens; 16 x 2), as one CTA serves it
+    for causal in (True, False):
+        for (g, Nq, Nk) in ((8, 4, 6), (16, 2, 9)):
+            q, k, v = rand((1, g, Nq, 3), 57), rand((1, 1, Nk, 3), 58), rand((1, 1, Nk, 3), 59)
+            o, lse = dec(q, k, v, causal, scale)
+            for h in range(g):
+                ob, lb = oracle.decode_naive_loops(q[0, h].tolist(), k[0, 0].tolist(), v[0, 0].tolist(), causal, scale)
+                np.testing.assert_allclose(o[0, h], np.array(ob), rtol=1e-12, atol=1e-12)
+                np.testing.assert_allclose(lse[0, h], np.array(lb), rtol=1e-12, atol=1e-12)
     # Nq = Nk is the square attention; the last Nq rows of a causal sequence are a causal decode
     N, d = 37, 8
     q, k, v = rand((2, 2, N, d), 54), rand((2, 1, N, d), 55), rand((2, 1, N, d), 56)
