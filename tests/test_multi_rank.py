@@ -77,10 +77,11 @@ def test_head_shards_cover_every_group_once():
             assert max(sizes) - min(sizes) <= 1
 
 
-def _shard_rank(rank, world, port, out):
+def _shard_rank(rank, world, port, out, kind="fwd"):
     """Each rank computes its head slice as an independent problem (B = 1) with
     the float64 oracle standing in for the kernel, then all ranks gather the
-    slices: the result must equal the unsharded problem."""
+    slices: the result must equal the unsharded problem. kind "decode": a few
+    new queries per head against a longer key/value cache."""
     import datetime
     import sys
 
@@ -93,28 +94,31 @@ def _shard_rank(rank, world, port, out):
     import exact_io_aware_44_b200 as fa
     import oracle
     B, Hq, Hkv, N, d = 3, 8, 2, 19, 8
+    Nq = 3 if kind == "decode" else N
     rng = np.random.default_rng(7)
-    q, k, v = rng.standard_normal((B, Hq, N, d)), rng.standard_normal((B, Hkv, N, d)), rng.standard_normal((B, Hkv, N, d))
+    q, k, v = rng.standard_normal((B, Hq, Nq, d)), rng.standard_normal((B, Hkv, N, d)), rng.standard_normal((B, Hkv, N, d))
+    fn = oracle.decode_fwd64 if kind == "decode" else oracle.attention_fwd64
     q0, q1, k0, k1 = fa.head_shard(B, Hq, Hkv, rank, world)
-    qs = q.reshape(B * Hq, N, d)[q0:q1][None]
+    qs = q.reshape(B * Hq, Nq, d)[q0:q1][None]
     ks = k.reshape(B * Hkv, N, d)[k0:k1][None]
     vs = v.reshape(B * Hkv, N, d)[k0:k1][None]
-    o, lse = oracle.attention_fwd64(qs, ks, vs, True, 0.3)
+    o, lse = fn(qs, ks, vs, True, 0.3)
     parts = [None] * world
     dist.all_gather_object(parts, (q0, q1, o[0], lse[0]))
-    full_o = np.concatenate([p[2] for p in sorted(parts, key=lambda p: p[0])]).reshape(B, Hq, N, d)
-    full_l = np.concatenate([p[3] for p in sorted(parts, key=lambda p: p[0])]).reshape(B, Hq, N)
-    ref_o, ref_l = oracle.attention_fwd64(q, k, v, True, 0.3)
+    full_o = np.concatenate([p[2] for p in sorted(parts, key=lambda p: p[0])]).reshape(B, Hq, Nq, d)
+    full_l = np.concatenate([p[3] for p in sorted(parts, key=lambda p: p[0])]).reshape(B, Hq, Nq)
+    ref_o, ref_l = fn(q, k, v, True, 0.3)
     out.put((rank, float(np.abs(full_o - ref_o).max()), float(np.abs(full_l - ref_l).max())))
     dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_head_sharded_problem_equals_the_whole():
+@pytest.mark.parametrize("kind", ["fwd", "decode"])
+def test_two_gloo_ranks_head_sharded_problem_equals_the_whole(kind):
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_shard_rank, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_shard_rank, args=(r, world, port, q, kind)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
