@@ -36,6 +36,11 @@
  *             never traps or spins forever.
  *   Sizes     B, Hq, Hkv >= 1; N >= 0 (N == 0 is a no-op that returns FA_OK);
  *             B*Hq*N < 2^31.
+ *   Contexts  The library caches, per device, the device addresses of its own
+ *             __device__ variables (the status word, fa_bwd_noalloc's scratch)
+ *             on first use. cudaDeviceReset() destroys the context those
+ *             addresses belong to: do not call into the library on a device
+ *             after resetting it in the same process.
  */
 #ifndef FA_B200_H_
 #define FA_B200_H_
