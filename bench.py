@@ -58,8 +58,9 @@ NCU_TRAFFIC = {
 # to end marker) plus the shared device helpers. Edits elsewhere in the file (the
 # other head-dim variant, comments) leave the recorded counters valid.
 KERNEL_SOURCES = {
-    "bwd_main": ("fa_bwd_sm100.cu", [("__device__ __forceinline__ void red_add_v4", "// ----"),
-                                     ("struct Bwd128Cfg {", "int sm_count() {")]),
+    "bwd_main": ("fa_bwd_sm100.cu", [("__device__ __forceinline__ void red_add(", "// ----"),
+                                     ("struct Bwd128Cfg {", "struct Bwd64Cfg {")]),
+    "bwd_main_d64": ("fa_bwd_sm100.cu", [("struct Bwd64Cfg {", "cudaError_t launch_main_d128(")]),
     "fwd": ("fa_fwd_sm100.cu", [("", None)]),
     "decode_split": ("fa_decode_sm100.cu", [("template <int R>\nstruct DecCfg {", "template <int R>\ncudaError_t launch_decode_r(")]),
 }
@@ -130,61 +131,110 @@ def job_throughput(flops_per_step_per_rank: float, world: int, max_seconds_per_s
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons sampled every `interval_ms` by a
+    host thread through NVML while the timed region runs. `mark(True)` /
+    `mark(False)` bracket the region; the summary uses the samples inside it
+    (falling back to all samples when the region is shorter than one period).
+    Without NVML it falls back to `nvidia-smi -lms`. It only reads settings."""
 
-    def __init__(self, gpu_index: int, interval_ms: int = 100):
-        self.gpu = gpu_index
-        self.interval = interval_ms
-        self.proc = None
-        self.path = None
+    REASONS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, cuda_index: int, interval_ms: int = 10):
+        self.cuda_index = cuda_index
+        self.interval = interval_ms / 1000.0
+        self.samples = []      # (t, sm_mhz, max_mhz, power_w, reasons bitmask)
+        self.window = [None, None]
+        self._stop = None
+        self._thread = None
+        self._smi = None
+
+    def _handle(self, nv):
+        import torch
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
+
+    def _poll(self, nv, h):
+        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), mx,
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(reasons_fn(h))))
+            except Exception:
+                pass
+            self._stop.wait(self.interval)
 
     def __enter__(self):
-        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
-        os.close(fd)
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 f"-lms={self.interval}"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
-        time.sleep(0.3)
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self._stop = threading.Event()
+            self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
+            self._start_smi()
+        time.sleep(0.05)
         return self
 
+    def _start_smi(self):
+        fields = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.sw_power_cap,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown")
+        fd, path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self._smi = (subprocess.Popen(["nvidia-smi", f"--id={self.cuda_index}", f"--query-gpu={fields}",
+                                           "--format=csv,noheader,nounits", "-lms=20"],
+                                          stdout=open(path, "w"), stderr=subprocess.DEVNULL), path)
+        except OSError:
+            self._smi = None
+
+    def mark(self, start: bool):
+        self.window[0 if start else 1] = time.perf_counter()
+
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        time.sleep(0.02)
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        if self._smi is not None:
+            proc, path = self._smi
+            proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
+                proc.kill()
+            for r in csv.reader(io.StringIO(open(path).read())):
+                try:
+                    bits = sum(bit for (name, bit), val in zip(self.REASONS[:4], r[3:7])
+                               if val.strip().lower() == "active")
+                    self.samples.append((None, float(r[0]), float(r[1]), float(r[2]), bits))
+                except (ValueError, IndexError):
+                    continue
+            os.unlink(path)
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
-        rows = list(csv.reader(io.StringIO(open(self.path).read())))
-        os.unlink(self.path)
-        sm, mx, power, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            if len(r) < 9:
-                continue
-            try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
-                power.append(float(r[3]))
-            except ValueError:
-                continue
-            for name, val in zip(names, r[5:9]):
-                if val.strip().lower() == "active":
-                    reasons.add(name)
-        if not sm:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock samples"]}
-        # samples under load: power well above idle
-        hi = [s for s, p in zip(sm, power) if p >= 0.5 * max(power)] or sm
-        return {"sm_mhz": statistics.median(hi), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm), "power_w_max": max(power)}
+        t0, t1 = self.window
+        inside = [s for s in self.samples if s[0] is not None and t0 is not None and t1 is not None
+                  and t0 <= s[0] <= t1]
+        used = inside if len(inside) >= 3 else self.samples
+        sm = [s[1] for s in used]
+        reasons = sorted({name for s in used for name, bit in self.REASONS if s[4] & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(s[2] for s in used), "sm_mhz_min": min(sm),
+                "reasons": reasons, "samples": len(used),
+                "window": "timed region" if used is inside else "whole sampler run (region shorter than 3 periods)",
+                "interval_ms": round(self.interval * 1000), "power_w_max": max(s[3] for s in used),
+                "source": "nvml" if self._thread is not None else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
@@ -331,11 +381,13 @@ def run_ours(args, w, world, rank, local):
         torch.cuda.synchronize()
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
+        clocks.mark(True)
         t_start.record(stream)
         for i in range(K):
             step(evs[i])
         t_end.record(stream)
         torch.cuda.synchronize()
+        clocks.mark(False)
         barrier()
     st = fa.get_status()
     if st:
@@ -360,9 +412,12 @@ def run_ours(args, w, world, rank, local):
     }
     dominant = max(("fwd", "bwd_main"), key=lambda k: kernels[k]["ms"])
     achieved = kernels[dominant]["tflops"]
+    dom_ms_med = statistics.median(per_kernel[dominant])
+    achieved_med = (f_fwd if dominant == "fwd" else f_bwd) / dom_ms_med / 1e9
     traffic = None
+    src_name = "bwd_main_d64" if (dominant == "bwd_main" and d == 64) else dominant
     rec = NCU_TRAFFIC.get((dominant, w.name))
-    if rec and rec.get("csrc_sha") == kernel_source_hash(dominant):
+    if rec and rec.get("csrc_sha") == kernel_source_hash(src_name):
         traffic = rec["bytes_per_launch"]
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": UNIT,
                 "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": dominant,
@@ -370,7 +425,9 @@ def run_ours(args, w, world, rank, local):
                                 if peak_src == "measured" else "fallback 1.59 PFLOP/s")
                 + (" x 2, the nominal dense fp8:bf16 ratio" if fp8 else ""),
                 "frac_of_sustained": round(achieved / (float(peaks.get("bf16_tflops_sustained", peak)) * peak_mul),
-                                           4)}
+                                           4),
+                # achieved/frac above use the mean launch time over the timed steps; these the median
+                "achieved_median": round(achieved_med, 1), "frac_median": round(achieved_med / peak, 4)}
 
     # ---------------------------------------------------- end to end (host buffers)
     # Through the public C ABI, every step uploads its inputs from pinned host memory
@@ -496,6 +553,9 @@ def run_ours(args, w, world, rank, local):
         "kernels_ms": {k: round(v["ms"], 4) for k, v in kernels.items()},
         "kernels_ms_median_min": {k: [round(statistics.median(v), 4), round(min(v), 4)]
                                   for k, v in per_kernel.items() if (w.backward or k == "fwd")},
+        # first timed step and slowest step per kernel: where a mean above the median comes from
+        "kernels_ms_first_max": {k: [round(v[0], 4), round(max(v), 4)]
+                                 for k, v in per_kernel.items() if (w.backward or k == "fwd")},
         # The pages' traffic argument: standard attention writes the N x N scores and
         # reads them back (fp16 S and P, each written and read once: 8 B*Hq*N^2 bytes);
         # this path moves only the O(N) tensors (algorithmic bytes; ncu-measured DRAM
@@ -513,7 +573,140 @@ def run_ours(args, w, world, rank, local):
         "gpu_launches": (4 if w.backward else 1) * K,
         "clocks": clk,
     }
+    if w.name == "c3" and world == 1 and args.shard != "heads" and not args.no_extras:
+        result["other_configs"] = other_configs(args, fa, torch, dev, stream, peak)
     return result
+
+
+def other_configs(args, fa, torch, dev, stream, peak):
+    """The remaining workloads the utilisation targets name, timed after the main
+    line on the same device: the c4 forward, the c5 forward and backward, the c2
+    (d = 64) forward and backward, and one decode step. Same timing as the main
+    line: CUDA events around each launch on the launching stream, after warm-up,
+    no parity work inside. Inputs: c4, c5 and dec are drawn on the device by a
+    seeded torch generator with the workloads' distributions (iid N(0, 1)), since
+    they are larger than L2 and drawing them on the host would dominate the run;
+    c2 uses the parity tests' seeded host recipe (with its spiked rows) and, being
+    smaller than L2, a 512 MB buffer is overwritten before every timed launch."""
+    import synth
+    sp = stream.cuda_stream
+    P = lambda t: t.data_ptr()
+    K = max(5, min(args.steps, 20))
+    Wm = max(3, args.warmup)
+    gen = torch.Generator(device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    out = {}
+
+    def timed(launches, n_events, l2_flush):
+        """Run `launches(events)` Wm + K times; returns per-interval lists of ms."""
+        for _ in range(Wm):
+            launches(None)
+        torch.cuda.synchronize()
+        rec = []
+        for _ in range(K):
+            if l2_flush:
+                flush.fill_(1)
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
+            launches(evs)
+            rec.append(evs)
+        torch.cuda.synchronize()
+        st = fa.get_status()
+        if st:
+            raise fa.FAError(st, "other configs")
+        return [[r[i].elapsed_time(r[i + 1]) for r in rec] for i in range(n_events - 1)]
+
+    def entry(wname, shape, ms_lists, names, f_fwd, f_bwd, inputs):
+        e = {"shape": shape, "inputs": inputs, "steps": K, "warmup": Wm}
+        med = {n: statistics.median(v) for n, v in zip(names, ms_lists)}
+        e["ms_median"] = {n: round(v, 4) for n, v in med.items()}
+        e["fwd_tflops"] = round(f_fwd / med["fwd"] / 1e9, 1)
+        e["fwd_pct_of_peak"] = round(100 * f_fwd / med["fwd"] / 1e9 / peak, 2)
+        if f_bwd:
+            bwd_ms = med["bwd_preprocess"] + med["bwd_main"] + med["bwd_convert"]
+            e["bwd_tflops"] = round(f_bwd / bwd_ms / 1e9, 1)
+            e["bwd_pct_of_peak"] = round(100 * f_bwd / bwd_ms / 1e9 / peak, 2)
+            e["bwd_main_tflops"] = round(f_bwd / med["bwd_main"] / 1e9, 1)
+            e["bwd_main_frac"] = round(f_bwd / med["bwd_main"] / 1e9 / peak, 4)
+        out[wname] = e
+
+    def attn(wl, tensors, inputs, l2_flush):
+        B, Hq, Hkv, N, d = wl.B, wl.Hq, wl.Hkv, wl.N, wl.d
+        q, k, v = tensors[:3]
+        o = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+        if wl.backward:
+            do = tensors[3]
+            dq, dk, dv = torch.empty_like(o), torch.empty_like(k), torch.empty_like(v)
+            ws = torch.empty(fa.workspace_bytes(B, Hq, Hkv, N, d), dtype=torch.uint8, device=dev)
+
+        def launches(evs):
+            if evs is not None:
+                evs[0].record(stream)
+            rc = fa.fwd_raw(P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, wl.causal, wl.scale, sp)
+            if rc:
+                raise fa.FAError(rc, "fa_fwd")
+            if evs is not None:
+                evs[1].record(stream)
+            if wl.backward:
+                between = (lambda i: evs[1 + i].record(stream)) if evs is not None else None
+                rc = fa.bwd_phases_raw(P(q), P(k), P(v), P(o), P(lse), P(do), P(dq), P(dk), P(dv), P(ws), B, Hq,
+                                       Hkv, N, d, wl.causal, wl.scale, sp, between=between)
+                if rc:
+                    raise fa.FAError(rc, "fa_bwd")
+
+        names = ("fwd", "bwd_preprocess", "bwd_main", "bwd_convert") if wl.backward else ("fwd",)
+        ms = timed(launches, len(names) + 1, l2_flush)
+        shape = (f"B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} {'causal' if wl.causal else 'non-causal'} bf16 "
+                 f"{'fwd+bwd' if wl.backward else 'fwd'}")
+        entry(wl.name, shape, ms, names, wl.fwd_flops(), wl.bwd_flops() if wl.backward else 0.0, inputs)
+
+    def dev_randn(wl, tid, heads):
+        gen.manual_seed(wl.seed * 16 + tid)
+        x = torch.randn((wl.B, heads, wl.N, wl.d), generator=gen, device=dev, dtype=torch.float32)
+        return (x * wl.std).to(torch.bfloat16)
+
+    for name in ("c4", "c5"):
+        wl = synth.WORKLOADS[name]
+        ts = [dev_randn(wl, tid, wl.Hq if tid in (synth.TID_Q, synth.TID_DO) else wl.Hkv)
+              for tid in ((synth.TID_Q, synth.TID_K, synth.TID_V) + ((synth.TID_DO,) if wl.backward else ()))]
+        attn(wl, ts, "seeded torch.randn on the device, iid N(0,1), rounded to bf16", False)
+        del ts
+    wl = synth.WORKLOADS["c2"]
+    ts = [torch.from_numpy(synth.tensor(wl, tid)).to(dev, torch.bfloat16)
+          for tid in (synth.TID_Q, synth.TID_K, synth.TID_V, synth.TID_DO)]
+    attn(wl, ts, "the parity tests' seeded host recipe (1% of query rows x20); L2 overwritten before each step",
+         True)
+    del ts
+    # decode: one new query per head against a 32768-key cache
+    dw = synth.DECODE_WORKLOADS["dec"]
+    gen.manual_seed(dw.seed)
+    qd = torch.randn((dw.B, dw.Hq, dw.Nq, dw.d), generator=gen, device=dev).to(torch.bfloat16)
+    kd = torch.randn((dw.B, dw.Hkv, dw.Nk, dw.d), generator=gen, device=dev).to(torch.bfloat16)
+    vd = torch.randn((dw.B, dw.Hkv, dw.Nk, dw.d), generator=gen, device=dev).to(torch.bfloat16)
+    od = torch.empty_like(qd)
+    ld = torch.empty((dw.B, dw.Hq, dw.Nq), dtype=torch.float32, device=dev)
+    wsd = torch.empty(fa.decode_workspace_bytes(dw.B, dw.Hq, dw.Hkv, dw.Nq, dw.Nk, dw.d), dtype=torch.uint8,
+                      device=dev)
+
+    def dec_launch(evs):
+        if evs is not None:
+            evs[0].record(stream)
+        rc = fa.decode_raw(P(qd), P(kd), P(vd), P(od), P(ld), P(wsd), dw.B, dw.Hq, dw.Hkv, dw.Nq, dw.Nk, dw.d,
+                           dw.causal, dw.scale, 0, sp)
+        if rc:
+            raise fa.FAError(rc, "fa_decode")
+        if evs is not None:
+            evs[1].record(stream)
+
+    ms = statistics.median(timed(dec_launch, 2, False)[0])
+    peaks, _ = load_peaks()
+    algo = dw.kv_bytes() + 2 * qd.numel() * 2 + ld.numel() * 4
+    out["dec"] = {"shape": f"decode B={dw.B} Hq={dw.Hq} Hkv={dw.Hkv} Nq={dw.Nq} Nk={dw.Nk} d={dw.d} causal bf16",
+                  "inputs": "seeded torch.randn on the device, iid N(0,1), rounded to bf16",
+                  "ms_median": round(ms, 4), "gbs": round(algo / ms / 1e6, 1),
+                  "frac_of_hbm": round(algo / ms / 1e6 / float(peaks["hbm_gbs"]), 4), "steps": K, "warmup": Wm}
+    del flush
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -584,11 +777,13 @@ def run_decode(args, w, world, rank, local):
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        clocks.mark(True)
         e0.record(stream)
         for _ in range(K):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
+        clocks.mark(False)
         barrier()
     if fa.get_status():
         raise fa.FAError(fa.get_status(), "timed region")
@@ -705,6 +900,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="c3: skip timing the other workloads (c4, c5, c2, dec) after the main line")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

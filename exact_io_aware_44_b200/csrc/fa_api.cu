@@ -18,6 +18,24 @@ namespace fa {
 // First device-side error since the last fa_get_status(); 0 = none.
 __device__ int g_status = 0;
 
+int sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 148;
+  }
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -104,6 +122,22 @@ int make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box_
   CUresult r = enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
+}
+
+// 3-D fp32 tensor map over the dQ accumulator [heads, N, d] with a 32-column
+// (128-byte), 128-row box and the 128-byte swizzle: the target of the d = 64
+// backward's TMA reduce-adds. Rows past N are never written.
+int make_map_acc(CUtensorMap* m, const float* base, int d, int N, int heads) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc) return FA_ERR_LAUNCH;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)N * d * 4};
+  cuuint32_t box[3] = {32, (cuuint32_t)kTileM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -395,7 +429,8 @@ int run_bwd(int phases, const void* q, const void* k, const void* v, const void*
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_ALIGNMENT;
   DeviceInfo* di;
   if ((rc = current_device(&di)) != FA_OK) return rc;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  memset(&tdq, 0, sizeof(tdq));
   if (main) {
     const int q_rows = bwd_query_rows(d);  // query rows per backward tile
     if ((rc = make_map(&tq, q, d, N, B * Hq, q_rows)) != FA_OK) return rc;
@@ -417,6 +452,7 @@ int run_bwd(int phases, const void* q, const void* k, const void* v, const void*
   p.dv = dv;
   p.delta = static_cast<float*>(workspace);
   p.dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + delta_bytes);
+  if (main && d == 64 && (rc = make_map_acc(&tdq, p.dq_acc, d, N, B * Hq)) != FA_OK) return rc;
   p.status = di->status;
   p.B = B;
   p.Hq = Hq;
@@ -431,7 +467,7 @@ int run_bwd(int phases, const void* q, const void* k, const void* v, const void*
   p.wait_budget_ns = g_wait_budget_ns.load();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (pre && launch_bwd_preprocess(p, s) != cudaSuccess) return FA_ERR_LAUNCH;
-  if (main && launch_bwd_main(tq, tk, tv, tdo, p, s) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (main && launch_bwd_main(tq, tk, tv, tdo, tdq, p, s) != cudaSuccess) return FA_ERR_LAUNCH;
   if (conv && launch_bwd_convert(p, s) != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
 }

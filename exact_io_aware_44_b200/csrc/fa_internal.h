@@ -86,10 +86,13 @@ cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 int bwd_query_rows(int d);
 // Backward phases: D and zeroed dQ accumulator; main kernel; dQ conversion.
 cudaError_t launch_bwd_preprocess(const BwdParams& p, cudaStream_t s);
+// `tdq`: fp32 map over the dQ accumulator (d = 64 only; 32-column, 128-row box, 128-byte swizzle).
 cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const BwdParams& p, cudaStream_t s);
+                            const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdParams& p, cudaStream_t s);
 cudaError_t launch_bwd_convert(const BwdParams& p, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* status, uint64_t budget_ns, cudaStream_t s);
+// Streaming multiprocessors of the current device (148 on a B200).
+int sm_count();
 
 // Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current device,
 // once per device (the attribute is per device; `done` holds one bit per device

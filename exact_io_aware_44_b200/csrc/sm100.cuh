@@ -131,6 +131,37 @@ __device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, con
   return false;
 }
 
+// How the many-thread consumer roles wait for a phase (all lanes of the warp call it
+// together; the result is the same on every lane):
+//   0  every lane polls with try_wait (suspending for at most kConsumerPollNs)
+//   1  every lane spins on test_wait
+//   2  lane 0 polls with try_wait, the others meet it at __syncwarp
+//   3  lane 0 spins on test_wait, the others meet it at __syncwarp
+// In modes 2 and 3 the warp barrier orders the other lanes after lane 0's acquire.
+#ifndef FA_CONSUMER_WAIT_MODE
+#define FA_CONSUMER_WAIT_MODE 0
+#endif
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, const WaitCtx& w);
+__device__ __forceinline__ bool consumer_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+#if FA_CONSUMER_WAIT_MODE == 0
+  return mbar_wait_ns(bar, parity, w, kConsumerPollNs);
+#elif FA_CONSUMER_WAIT_MODE == 1
+  return mbar_wait_spin(bar, parity, w);
+#else
+  bool ok = false;
+  if ((threadIdx.x & 31) == 0) {
+#if FA_CONSUMER_WAIT_MODE == 2
+    ok = mbar_wait_ns(bar, parity, w, kConsumerPollNs);
+#else
+    ok = mbar_wait_spin(bar, parity, w);
+#endif
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok;
+#endif
+}
+
 // Non-suspending probe of a phase (mbarrier.test_wait).
 __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -199,6 +230,33 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+
+// 3-D tiled reduction of one shared-memory box into global memory: every element
+// of the box is added (fp32 add, done by the TMA unit at L2) to the tensor at
+// (x, y, z). Elements outside the tensor's bounds are skipped. Tracked by the
+// issuing thread's bulk async-groups; the shared source must not be rewritten
+// before bulk_wait_read() says the unit has read it.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until every bulk group this thread committed has completed (writes done).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Barrier over `count` threads (a multiple of 32) on hardware barrier `id` (1..15;
+// 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ----------------------------------------------------------------------------

@@ -61,6 +61,26 @@ def test_bf16_fwd_small(cuda_device, shape, causal):
     check_full(w, cuda_device)
 
 
+# More work units (query blocks x heads) than SMs, so that each CTA of the
+# persistent grid runs several units in a row, among them units whose second
+# query tile lies past N (N = 800 and 300: the last block holds one tile).
+PERSISTENT_SHAPES = [
+    # B, Hq, Hkv, N, d
+    (2, 40, 8, 800, 64),
+    (2, 40, 8, 800, 128),
+    (1, 160, 160, 300, 256),
+    (3, 64, 16, 520, 128),
+]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("shape", PERSISTENT_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_bf16_fwd_many_units_per_cta(cuda_device, shape, causal):
+    B, Hq, Hkv, N, d = shape
+    w = synth.small(B, Hq, Hkv, N, d, causal, seed=1300 + N + d)
+    check_full(w, cuda_device)
+
+
 D256_SHAPES = [
     # B, Hq, Hkv, N (d = 256: one 128-row query tile per CTA)
     (1, 1, 1, 1),
