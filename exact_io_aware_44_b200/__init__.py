@@ -19,7 +19,7 @@ import math
 import os
 
 __all__ = ["head_shard", "fwd", "fwd_fp8", "decode", "decode_raw", "decode_workspace_bytes", "bwd", "fwd_raw", "fwd_fp8_raw", "bwd_raw", "bwd_phases_raw", "workspace_bytes", "get_status", "set_wait_budget_ns",
-           "selftest_wait_timeout", "FAError", "LIB_PATH", "lib", "STATUS"]
+           "selftest_wait_timeout", "get_progress", "FAError", "LIB_PATH", "lib", "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
 
@@ -44,6 +44,7 @@ SIGNATURES = {
     "fa_bwd_convert": (_I, [_P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_get_status": (_I, [_P]),
+    "fa_get_progress": (_I, [_P, _I, _P]),
     "fa_set_wait_budget_ns": (None, [ctypes.c_uint64]),
     "fa_selftest_wait_timeout": (_I, [ctypes.c_uint64, _P]),
     "fa_error_string": (ctypes.c_char_p, [_I]),
@@ -294,6 +295,16 @@ def bwd(q, k, v, o, lse, do, causal: bool = True, scale: float | None = None, wo
 def get_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return int(lib.fa_get_status(_stream_ptr(stream)))
+
+
+def get_progress(n: int, stream=None):
+    """Per-CTA progress words of the last forward / backward main-kernel launch
+    (see fa_get_progress in include/fa.h), as a list of n ints."""
+    buf = (ctypes.c_uint * max(int(n), 0))()
+    rc = lib.fa_get_progress(ctypes.cast(buf, ctypes.c_void_p), int(n), _stream_ptr(stream))
+    if rc < 0:
+        raise FAError(rc, "fa_get_progress")
+    return list(buf)[:rc]
 
 
 def set_wait_budget_ns(ns: int):

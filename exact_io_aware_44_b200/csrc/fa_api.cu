@@ -18,6 +18,10 @@ namespace fa {
 // First device-side error since the last fa_get_status(); 0 = none.
 __device__ int g_status = 0;
 
+// Progress record of the last forward / backward main-kernel launch on this device:
+// word i is how far CTA i got (see fa_get_progress).
+__device__ unsigned g_progress[kProgressSlots];
+
 int sm_count() {
   static std::atomic<int> cache[64];
   int dev = 0;
@@ -58,6 +62,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 struct DeviceInfo {
   int checked = 0;  // 0 = not yet, 1 = sm_100, -1 = not sm_100
   int* status = nullptr;
+  unsigned* progress = nullptr;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -86,6 +91,11 @@ int current_device(DeviceInfo** out) {
         return FA_ERR_LAUNCH;
       }
       di.status = static_cast<int*>(ptr);
+      if (cudaGetSymbolAddress(&ptr, g_progress) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+      }
+      di.progress = static_cast<unsigned*>(ptr);
       di.checked = 1;
     }
   }
@@ -215,6 +225,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_scale = 1.f;
   p.wait_budget_ns = g_wait_budget_ns.load();
+  p.progress = di->progress;
+  p.progress_n = kProgressSlots;
   if (launch_fwd_bf16(tq, tk, tv, p, d, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
 }
@@ -253,6 +265,8 @@ static int fwd_f8(bool e5m2, const void* q, const void* k, const void* v, float 
   p.scale_log2 = c;
   p.o_scale = descale_v;
   p.wait_budget_ns = g_wait_budget_ns.load();
+  p.progress = di->progress;
+  p.progress_n = kProgressSlots;
   const cudaError_t e = e5m2 ? launch_fwd_e5m2(tq, tk, tv, p, static_cast<cudaStream_t>(stream))
                              : launch_fwd_e4m3(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return FA_ERR_LAUNCH;
@@ -465,6 +479,8 @@ int run_bwd(int phases, const void* q, const void* k, const void* v, const void*
   // per kv head, for its Hq / Hkv query heads: Q and dO (bf16), the fp32 dQ accumulator, LSE and D
   p.head_group = head_group((double)(Hq / Hkv) * N * (8.0 * d + 8), 1, B * Hkv);
   p.wait_budget_ns = g_wait_budget_ns.load();
+  p.progress = di->progress;
+  p.progress_n = kProgressSlots;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (pre && launch_bwd_preprocess(p, s) != cudaSuccess) return FA_ERR_LAUNCH;
   if (main && launch_bwd_main(tq, tk, tv, tdo, tdq, p, s) != cudaSuccess) return FA_ERR_LAUNCH;
@@ -514,6 +530,21 @@ int fa_get_status(void* stream) {
   if (v != 0 && cudaMemcpy(di->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return FA_ERR_LAUNCH;
   return v;
+}
+
+int fa_get_progress(unsigned* out, int n, void* stream) {
+  if (!out || n < 0) return FA_ERR_INVALID_ARG;
+  if (n > kProgressSlots) n = kProgressSlots;
+  DeviceInfo* di;
+  int rc = current_device(&di);
+  if (rc != FA_OK) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  if (n > 0 && cudaMemcpy(out, di->progress, (size_t)n * sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  return n;
 }
 
 int fa_selftest_wait_timeout(uint64_t budget_ns, void* stream) {

@@ -17,8 +17,8 @@
 //                     P^T = 2^(S^T c - LSE_i log2 e), dS^T = P^T o (dP^T - D_i)
 //                     dV += P^T dO_i, dK += dS^T Q_i            (TMEM accumulators)
 //                     dQ_i partial -> TMEM, then added to the fp32 accumulator
-//                     with red.global.add.
-//                   Two variants, one per head dim: bwd_main_kernel<64> and
+//                     (d = 128: red.global.add; d = 64: TMA reduce-add).
+//                   Two variants, one per head dim: bwd_main_d64_kernel and
 //                   bwd_main_d128_kernel (described where each is defined).
 //   bwd_convert     dQ = bf16(scale * accumulator).
 //
@@ -28,8 +28,8 @@
 //   warp 1      allocates TMEM; one lane issues every tcgen05.mma.
 //   warps 4-11  two warpgroups, thread = key row; warpgroup h computes P^T and
 //               dS^T for query columns [64 h, 64 h + 64).
-//   warps 12-15 thread = TMEM lane of the dQ tile: reads it and issues the fp32
-//               reductions; at the end, writes dK and dV.
+//   warps 12-15 thread = TMEM lane of the dQ tile: reads it and adds it into the
+//               fp32 accumulator; at the end, writes dK and dV.
 #include <math.h>
 
 #include <algorithm>
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int h = kvh * g + it / per_head;
       const int i0 = (qt_first + it % per_head) * BR;
       const int q_head = b * p.Hq + h;
-      if (!(ok = mbar_wait_spin(&q_empty[s], use_par, w))) break;
+      if (!(ok = warp_wait_spin(&q_empty[s], use_par, w))) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(&q_full[s], C::kTile);
 #pragma unroll
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         dl[r] = in ? p.delta[rbase + i] : 0.f;
       }
       mbar_arrive(&q_full[s]);
-      if (!(ok = mbar_wait_spin(&do_empty[s], use_par, w))) break;
+      if (!(ok = warp_wait_spin(&do_empty[s], use_par, w))) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(&do_full[s], C::kTile);
 #pragma unroll
@@ -354,9 +354,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_bf16_ss(tmem + C::kColDQ, desc_advance(dK_mn, k * 2048), desc_advance(dS_mn, k * 2048), kIdQ,
                       k > 0 ? 1u : 0u);
     };
-    bool ok = mbar_wait_spin(kv_full, 0, w);
-    if (ok && n_it > 0) ok = mbar_wait_spin(&q_full[0], 0, w);
-    if (ok && n_it > 0) ok = mbar_wait_spin(&do_full[0], 0, w);
+    // progress record: the query tiles whose dV MMA this CTA has issued
+    unsigned* const prog = (int)blockIdx.x < p.progress_n ? p.progress : nullptr;
+    if (leader && prog) prog[blockIdx.x] = 0u;
+    bool ok = warp_wait_spin(kv_full, 0, w);
+    if (ok && n_it > 0) ok = warp_wait_spin(&q_full[0], 0, w);
+    if (ok && n_it > 0) ok = warp_wait_spin(&do_full[0], 0, w);
     tc_fence_after();
     if (ok && n_it > 0) {
       mma_scores(dK_k, dQ_k, C::kColS);
@@ -369,18 +372,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int s = it & 1;
       // dV += P^T dO_i, then S^T(i+1) into the columns P^T(i) came from (one
       // thread's MMAs execute in issue order)
-      if (!(ok = mbar_wait_spin(p_full, ph, w))) break;
+      if (!(ok = warp_wait_spin(p_full, ph, w))) break;
+      if (leader && prog) prog[blockIdx.x] = (unsigned)(it + 1);
       tc_fence_after();
       mma_dv(desc_advance(dDO_mn, s * C::kTile), it == 0);
       if (leader) mma_commit(&do_empty[s]);
       if (it + 1 < n_it) {
-        if (!(ok = mbar_wait_spin(&q_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
+        if (!(ok = warp_wait_spin(&q_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
         tc_fence_after();
         mma_scores(dK_k, desc_advance(dQ_k, (s ^ 1) * C::kTile), C::kColS);
         if (leader) mma_commit(s_full);
       }
       // dQ_i into the dP^T columns (already read), then dK += dS^T Q_i
-      if (!(ok = mbar_wait_spin(ds_full, ph, w))) break;
+      if (!(ok = warp_wait_spin(ds_full, ph, w))) break;
       tc_fence_after();
       mma_dq();
       if (leader) mma_commit(dq_full);
@@ -391,8 +395,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       // dP^T(i+1) once dQ_i has been read out of TMEM
       if (it + 1 < n_it) {
-        if (!(ok = mbar_wait_spin(dq_free, ph, w))) break;
-        if (!(ok = mbar_wait_spin(&do_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
+        if (!(ok = warp_wait_spin(dq_free, ph, w))) break;
+        if (!(ok = warp_wait_spin(&do_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
         tc_fence_after();
         mma_scores(dV_k, desc_advance(dDO_k, (s ^ 1) * C::kTile), C::kColDP);
         if (leader) mma_commit(dp_full);
@@ -442,11 +446,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       // P^T[key][q] = 2^(S c - LSE_q log2 e), zero for future queries and invalid keys.
       const uint64_t c2 = f2_pack(c, c);
-      const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2);
+      const ulonglong2* nl4 = reinterpret_cast<const ulonglong2*>(lse2);  // 16-byte broadcast loads
 #pragma unroll
       for (int i = 0; i < HB; i += 2) {
+        const ulonglong2 nv = nl4[i / 4];
         float x0, x1;
-        f2_unpack(f2_fma(f2_pack(pr[i], pr[i + 1]), c2, nl2[i / 2]), x0, x1);
+        f2_unpack(f2_fma(f2_pack(pr[i], pr[i + 1]), c2, (i & 2) ? nv.y : nv.x), x0, x1);
         if (((i / 2) & 7) < kBwdPolyPairs) {  // part of the exponentials on the FMA pipe
           ex2_poly2(x0, x1, pr[i], pr[i + 1]);
         } else {
@@ -473,24 +478,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(p_full);
-      // dS^T = P^T o (dP^T - D_q), 32 columns at a time
+      // dS^T = P^T o (dP^T - D_q); both halves of dP^T in flight before the one wait
       if (!consumer_wait(dp_full, ph, w)) break;
       tc_fence_after();
       uint32_t dsp[HB / 2];
-      const uint64_t* dl2 = reinterpret_cast<const uint64_t*>(dl);
+      const ulonglong2* dl4 = reinterpret_cast<const ulonglong2*>(dl);  // 16-byte broadcast loads
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tmem + lane_off + C::kColDP + col0, r0);
+        tmem_ld32(tmem + lane_off + C::kColDP + col0 + 32, r1);
+        tmem_ld_wait(r0);
+        tmem_ld_wait(r1);
 #pragma unroll
-      for (int cc = 0; cc < HB / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_off + C::kColDP + col0 + cc * 32, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int q = cc * 32 + i;
+        for (int i = 0; i < HB; i += 2) {
+          const uint32_t d0 = i < 32 ? r0[i] : r1[i - 32], d1 = i < 32 ? r0[i + 1] : r1[i - 31];
           float a, bb;
-          f2_unpack(f2_mul(f2_pack(pr[q], pr[q + 1]),
-                           f2_sub(f2_pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), dl2[q / 2])),
+          f2_unpack(f2_mul(f2_pack(pr[i], pr[i + 1]),
+                           f2_sub(f2_pack(__uint_as_float(d0), __uint_as_float(d1)),
+                                  (i & 2) ? dl4[i / 4].y : dl4[i / 4].x)),
                     a, bb);
-          dsp[q / 2] = pack_bf16x2(a, bb);
+          dsp[i / 2] = pack_bf16x2(a, bb);
         }
       }
       // the dS^T tile is free once dQ and dK of the previous query tile are done
@@ -734,7 +741,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int h = kvh * g + it / per_head;
       const int i0 = (qt_first + it % per_head) * BR;
       const int q_head = b * p.Hq + h;
-      if (!(ok = mbar_wait_spin(&q_empty[s], use_par, w))) break;
+      if (!(ok = warp_wait_spin(&q_empty[s], use_par, w))) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(&q_full[s], C::kTile);
         tma_load_3d(smem + C::kOffQ + s * C::kTile, &tmQ, &q_full[s], 0, i0, q_head);
@@ -750,7 +757,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         dl[rr] = in ? p.delta[rbase + i] : 0.f;
       }
       mbar_arrive(&q_full[s]);
-      if (!(ok = mbar_wait_spin(&do_empty[s], use_par, w))) break;
+      if (!(ok = warp_wait_spin(&do_empty[s], use_par, w))) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(&do_full[s], C::kTile);
         tma_load_3d(smem + C::kOffDO + s * C::kTile, &tmDO, &do_full[s], 0, i0, q_head);
@@ -807,9 +814,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_bf16_ss(tmem + col, desc_advance(dS_mn, k * 2048), desc_advance(dK_mn, k * 2048), kIdQ,
                       k > 0 ? 1u : 0u);
     };
-    bool ok = mbar_wait_spin(kv_full, 0, w);
-    if (ok && n_it > 0) ok = mbar_wait_spin(&q_full[0], 0, w);
-    if (ok && n_it > 0) ok = mbar_wait_spin(&do_full[0], 0, w);
+    // progress record: the query tiles whose dV MMA this CTA has issued
+    unsigned* const prog = (int)blockIdx.x < p.progress_n ? p.progress : nullptr;
+    if (leader && prog) prog[blockIdx.x] = 0u;
+    bool ok = warp_wait_spin(kv_full, 0, w);
+    if (ok && n_it > 0) ok = warp_wait_spin(&q_full[0], 0, w);
+    if (ok && n_it > 0) ok = warp_wait_spin(&do_full[0], 0, w);
     tc_fence_after();
     if (ok && n_it > 0) {
       mma_scores(dK_k, dQ_k, C::kColS);
@@ -821,19 +831,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t ph = it & 1;
       const int s = it & 1;
       const int qb = it & 1;  // dQ buffer
-      if (!(ok = mbar_wait_spin(p_full, ph, w))) break;
+      if (!(ok = warp_wait_spin(p_full, ph, w))) break;
+      if (leader && prog) prog[blockIdx.x] = (unsigned)(it + 1);
       tc_fence_after();
       mma_dv(desc_advance(dDO_mn, s * C::kTile), it == 0);
       if (leader) mma_commit(&do_empty[s]);
       if (it + 1 < n_it) {
-        if (!(ok = mbar_wait_spin(&q_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
+        if (!(ok = warp_wait_spin(&q_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
         tc_fence_after();
         mma_scores(dK_k, desc_advance(dQ_k, (s ^ 1) * C::kTile), C::kColS);
         if (leader) mma_commit(s_full);
       }
-      if (!(ok = mbar_wait_spin(ds_full, ph, w))) break;
+      if (!(ok = warp_wait_spin(ds_full, ph, w))) break;
       // the dQ buffer is free once dQ(it - 2) has been read out
-      if (it >= 2 && !(ok = mbar_wait_spin(&dq_free[qb], ((it >> 1) & 1) ^ 1, w))) break;
+      if (it >= 2 && !(ok = warp_wait_spin(&dq_free[qb], ((it >> 1) & 1) ^ 1, w))) break;
       tc_fence_after();
       mma_dq(C::kColDQ + qb * 64);
       if (leader) mma_commit(&dq_full[qb]);
@@ -843,7 +854,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_commit(ds_free);
       }
       if (it + 1 < n_it) {
-        if (!(ok = mbar_wait_spin(&do_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
+        if (!(ok = warp_wait_spin(&do_full[s ^ 1], ((it + 1) >> 1) & 1, w))) break;
         tc_fence_after();
         mma_scores(dV_k, desc_advance(dDO_k, (s ^ 1) * C::kTile), C::kColDP);
         if (leader) mma_commit(dp_full);
@@ -893,11 +904,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       // P^T[key][q] = 2^(S c - LSE_q log2 e), zero for future queries and invalid keys.
       const uint64_t c2 = f2_pack(c, c);
-      const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(lse2);
+      const ulonglong2* nl4 = reinterpret_cast<const ulonglong2*>(lse2);  // 16-byte broadcast loads
 #pragma unroll
       for (int i = 0; i < HB; i += 2) {
+        const ulonglong2 nv = nl4[i / 4];
         float x0, x1;
-        f2_unpack(f2_fma(f2_pack(pr[i], pr[i + 1]), c2, nl2[i / 2]), x0, x1);
+        f2_unpack(f2_fma(f2_pack(pr[i], pr[i + 1]), c2, (i & 2) ? nv.y : nv.x), x0, x1);
         pr[i] = ex2(x0);
         pr[i + 1] = ex2(x1);
       }
@@ -924,7 +936,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!consumer_wait(dp_full, ph, w)) break;
       tc_fence_after();
       uint32_t dsp[HB / 2];
-      const uint64_t* dl2 = reinterpret_cast<const uint64_t*>(dl);
+      const ulonglong2* dl4 = reinterpret_cast<const ulonglong2*>(dl);  // 16-byte broadcast loads
       {
         uint32_t r0[32], r1[32];
         tmem_ld32(tmem + lane_off + C::kColDP + col0, r0);
@@ -936,7 +948,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const uint32_t d0 = i < 32 ? r0[i] : r1[i - 32], d1 = i < 32 ? r0[i + 1] : r1[i - 31];
           float a, bb;
           f2_unpack(f2_mul(f2_pack(pr[i], pr[i + 1]),
-                           f2_sub(f2_pack(__uint_as_float(d0), __uint_as_float(d1)), dl2[i / 2])),
+                           f2_sub(f2_pack(__uint_as_float(d0), __uint_as_float(d1)),
+                                  (i & 2) ? dl4[i / 4].y : dl4[i / 4].x)),
                     a, bb);
           dsp[i / 2] = pack_bf16x2(a, bb);
         }

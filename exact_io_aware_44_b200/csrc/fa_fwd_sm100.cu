@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int cnt = 0;
     auto take = [&](int& slot) -> bool {  // next stage of the ring
       slot = cnt % S;
-      const bool res = mbar_wait_spin(&ring_full[slot], (cnt / S) & 1, w);
+      const bool res = warp_wait_spin(&ring_full[slot], (cnt / S) & 1, w);
       ++cnt;
       tc_fence_after();
       return res;
@@ -320,16 +320,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     };
     int p_base[2] = {0, 0};  // p_ready phases completed in earlier units, per tile
+    // progress record: the P V products this CTA has issued (both tiles, all its units)
+    unsigned* const prog = (int)blockIdx.x < p.progress_n ? p.progress : nullptr;
+    unsigned pv_count = 0;
+    if (leader && prog) prog[blockIdx.x] = 0u;
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int u = fwd_unit_index(k, n_units);
       if (u >= n_units) break;
       const FwdUnit U = fwd_unit<C::kTiles>(p, u);
-      if (!(ok = mbar_wait_spin(q_full, k & 1, w))) break;
+      if (!(ok = warp_wait_spin(q_full, k & 1, w))) break;
       tc_fence_after();
       {
         int kslot;
         if (!(ok = take(kslot))) break;
+#pragma unroll
         for (int t = 0; t < 2; ++t)
           if (U.n_iter[t] > 0) issue_s(t, kslot);
         if (leader) {
@@ -340,9 +345,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int j = 0; j < U.n_kv && ok; ++j) {
         int vslot, kslot = -1;
         if (!(ok = take(vslot))) break;
-        for (int t = 0; t < 2 && ok; ++t) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {  // unrolled: t, the TMEM columns and barriers are constants
           if (j >= U.n_iter[t]) continue;
-          if (!(ok = mbar_wait_spin(&p_ready[t], (p_base[t] + j) & 1, w))) break;
+          if (!(ok = warp_wait_spin(&p_ready[t], (p_base[t] + j) & 1, w))) break;
+          if (leader && prog) prog[blockIdx.x] = (unsigned)(++pv_count);
           tc_fence_after();
           issue_pv(t, vslot, j);
           if (j + 1 < U.n_iter[t]) {

@@ -24,6 +24,8 @@ struct FwdParams {
   float scale_log2;   // scale * log2(e) (times the Q and K descales for E4M3 inputs)
   float o_scale;      // multiplies O at the end (the V descale for E4M3 inputs, else 1)
   uint64_t wait_budget_ns;
+  unsigned* progress;  // per-CTA progress record (blockIdx.x < progress_n), or null
+  int progress_n;
 };
 
 struct FwdF32Params {
@@ -48,6 +50,8 @@ struct BwdParams {
   float scale_log2;
   int head_group;    // consecutive (batch, kv head) pairs scheduled together
   uint64_t wait_budget_ns;
+  unsigned* progress;  // per-CTA progress record (blockIdx.x < progress_n), or null
+  int progress_n;
 };
 
 struct DecodeParams {
@@ -93,6 +97,8 @@ cudaError_t launch_bwd_convert(const BwdParams& p, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* status, uint64_t budget_ns, cudaStream_t s);
 // Streaming multiprocessors of the current device (148 on a B200).
 int sm_count();
+// Slots of the per-CTA progress record: CTAs with blockIdx.x below this record.
+constexpr int kProgressSlots = 1 << 16;
 
 // Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current device,
 // once per device (the attribute is per device; `done` holds one bit per device

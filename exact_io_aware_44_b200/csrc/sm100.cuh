@@ -137,16 +137,20 @@ __device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, con
 //   1  every lane spins on test_wait
 //   2  lane 0 polls with try_wait, the others meet it at __syncwarp
 //   3  lane 0 spins on test_wait, the others meet it at __syncwarp
+//   4  every lane probes with test_wait and sleeps kConsumerPollNs between probes
 // In modes 2 and 3 the warp barrier orders the other lanes after lane 0's acquire.
 #ifndef FA_CONSUMER_WAIT_MODE
 #define FA_CONSUMER_WAIT_MODE 0
 #endif
 __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, const WaitCtx& w);
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, const WaitCtx& w, uint32_t ns);
 __device__ __forceinline__ bool consumer_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
 #if FA_CONSUMER_WAIT_MODE == 0
   return mbar_wait_ns(bar, parity, w, kConsumerPollNs);
 #elif FA_CONSUMER_WAIT_MODE == 1
   return mbar_wait_spin(bar, parity, w);
+#elif FA_CONSUMER_WAIT_MODE == 4
+  return mbar_wait_sleep(bar, parity, w, kConsumerPollNs);
 #else
   bool ok = false;
   if ((threadIdx.x & 31) == 0) {
@@ -188,6 +192,43 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, c
   for (uint64_t i = 0; i < max_iter; ++i) {
     if (mbar_test_wait(a, parity)) return true;
     if ((i & 63) == 63) {
+      if (*w.abort_flag) return false;
+      if (globaltimer_ns() - t0 > w.budget_ns) break;
+    }
+  }
+  *w.abort_flag = 1;
+  record_error(w.status, FA_ERR_DEVICE_TIMEOUT);
+  return false;
+}
+
+// A whole warp waits for a phase on behalf of one lane (MMA issuer, producer): with
+// FA_WARP_SPIN_LANE0 only lane 0 polls and the others meet it at the shuffle;
+// otherwise every lane polls. Every lane of the warp must call it; the result is
+// the same on all lanes.
+#ifndef FA_WARP_SPIN_LANE0
+#define FA_WARP_SPIN_LANE0 0
+#endif
+__device__ __forceinline__ bool warp_wait_spin(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+#if FA_WARP_SPIN_LANE0
+  bool ok = false;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_spin(bar, parity, w);
+  return __shfl_sync(0xffffffffu, ok, 0);
+#else
+  return mbar_wait_spin(bar, parity, w);
+#endif
+}
+
+// As mbar_wait_spin, with a nanosleep of about `ns` between probes, which gives the
+// issue slots back to the other warps of the sub-partition while waiting.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, const WaitCtx& w, uint32_t ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_test_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t max_iter = w.budget_ns / 8 + 1024;  // every probe takes well over 8 ns
+  for (uint64_t i = 0; i < max_iter; ++i) {
+    __nanosleep(ns);
+    if (mbar_test_wait(a, parity)) return true;
+    if ((i & 15) == 15) {
       if (*w.abort_flag) return false;
       if (globaltimer_ns() - t0 > w.budget_ns) break;
     }

@@ -249,6 +249,20 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
  */
 int fa_get_status(void* stream);
 
+/* fa_get_progress -- where each CTA of the last forward or backward main-kernel
+ * launch on the current device got to: a diagnostic for a launch that reported
+ * FA_ERR_DEVICE_TIMEOUT (the failure-detection side of the bounded waits; the
+ * pages describe no such record). Word i belongs to CTA i: for the forward, the
+ * number of P V products CTA i had issued (both of its query tiles, every work
+ * unit it ran); for the backward main kernel, the number of query tiles whose
+ * dV += P^T dO it had issued. Each CTA sets its word to 0 when it starts; words
+ * of CTAs that did not run in the last launch keep older values. CTAs with index
+ * 65536 or more keep no record.
+ *   out     host buffer of n unsigned words; n is clamped to 65536.
+ * Synchronises `stream`, then copies. Returns the number of words copied, or a
+ * negative fa_status_t (FA_ERR_INVALID_ARG for a null buffer or n < 0). */
+int fa_get_progress(unsigned* out, int n, void* stream);
+
 /* fa_set_wait_budget_ns -- budget of each bounded device-side wait (default
  * 2e9 ns). Kernels launched afterwards use the new value. Values outside
  * [1e5, 6e10] ns are clamped to that range. */

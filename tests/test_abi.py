@@ -149,3 +149,10 @@ def test_no_device_is_reported_without_gpu():
         pytest.skip("a GPU is present")
     assert _fwd() == -6
     assert fa.lib.fa_get_status(None) == -6
+
+
+def test_progress_record_rejects_bad_arguments_on_host():
+    import ctypes
+    buf = (ctypes.c_uint * 4)()
+    assert fa.lib.fa_get_progress(None, 4, None) == -1
+    assert fa.lib.fa_get_progress(ctypes.cast(buf, ctypes.c_void_p), -1, None) == -1

@@ -225,3 +225,21 @@ def test_bounded_wait_reports_timeout(cuda_device):
     import exact_io_aware_44_b200 as fa
     assert fa.selftest_wait_timeout(5_000_000) == -5
     assert fa.get_status() == 0   # the status word was cleared
+
+
+def test_progress_record_counts_each_ctas_work(cuda_device):
+    """The per-CTA progress words after a launch equal the work each CTA was
+    given: P V products in the forward, query tiles in the backward."""
+    import torch
+    import exact_io_aware_44_b200 as fa
+    w = synth.small(1, 2, 1, 300, 128, True, seed=4)
+    q, k, v, do = (to_dev(synth.tensor(w, t), torch.bfloat16, cuda_device)
+                   for t in (synth.TID_Q, synth.TID_K, synth.TID_V, synth.TID_DO))
+    o, lse = fa.fwd(q, k, v, causal=True)
+    # 2 heads x 2 blocks of 256 query rows; each block issues 3 P V products
+    # (rows 0-255: 1 + 2 key tiles; rows 256-299: 3 key tiles)
+    assert fa.get_progress(4) == [3, 3, 3, 3]
+    fa.bwd(q, k, v, o, lse, do, causal=True)
+    # key tiles 0, 1, 2 of the one kv head see 3, 2, 1 query tiles of each of 2 query heads
+    assert sorted(fa.get_progress(3)) == [2, 4, 6]
+    assert fa.get_status() == 0
