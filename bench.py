@@ -47,10 +47,15 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 # source makes the figure stale and the bench reports null.
 NCU_TRAFFIC = {
     # profiles/bwd_main_d128_B2H32N8192_causal.md
-    ("bwd_main", "c3"): {"bytes_per_launch": 810462464 + 489935104, "csrc_sha": "ed7fc08fb60db3a8"},
+    ("bwd_main", "c3"): {"bytes_per_launch": 810287616 + 489886208, "csrc_sha": "1896da15478db7ec"},
+    # profiles/bwd_main_d64_B4H16N2048_causal.md (--set full capture)
+    ("bwd_main", "c2"): {"bytes_per_launch": 101763584 + 22738176, "csrc_sha": "56c56e7e3931d08b"},
+    # profiles/fwd_bf16_d128_B2H32N8192_causal.md
+    ("fwd", "c3"): {"bytes_per_launch": 404763136 + 118222336, "csrc_sha": "6850015faac09dea"},
+    ("fwd", "c4"): {"bytes_per_launch": 810670592 + 261153792, "csrc_sha": "6850015faac09dea"},
     # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md
-    ("decode_split", "dec"): {"bytes_per_launch": 2148211200 + 3646464, "csrc_sha": "23e740588e569a93"},
-    ("decode_split", "dec4"): {"bytes_per_launch": 1074812160 + 4330240, "csrc_sha": "23e740588e569a93"},
+    ("decode_split", "dec"): {"bytes_per_launch": 2148272896 + 3852544, "csrc_sha": "4137ec07188f1845"},
+    ("decode_split", "dec4"): {"bytes_per_launch": 1074823168 + 4116480, "csrc_sha": "4137ec07188f1845"},
 }
 
 
@@ -595,28 +600,39 @@ def other_configs(args, fa, torch, dev, stream, peak):
     Wm = max(3, args.warmup)
     gen = torch.Generator(device=dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    peaks_all, _ = load_peaks()
+    peak_sustained = float(peaks_all.get("bf16_tflops_sustained", peak))
     out = {}
 
+    last_clocks = {}
+
     def timed(launches, n_events, l2_flush):
-        """Run `launches(events)` Wm + K times; returns per-interval lists of ms."""
+        """Run `launches(events)` Wm + K times; returns per-interval lists of ms. The
+        clocks seen during the K timed runs are left in last_clocks."""
         for _ in range(Wm):
             launches(None)
         torch.cuda.synchronize()
         rec = []
-        for _ in range(K):
-            if l2_flush:
-                flush.fill_(1)
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
-            launches(evs)
-            rec.append(evs)
-        torch.cuda.synchronize()
+        with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+            clocks.mark(True)
+            for _ in range(K):
+                if l2_flush:
+                    flush.fill_(1)
+                evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
+                launches(evs)
+                rec.append(evs)
+            torch.cuda.synchronize()
+            clocks.mark(False)
+        last_clocks.clear()
+        last_clocks.update(clocks.summary())
         st = fa.get_status()
         if st:
             raise fa.FAError(st, "other configs")
         return [[r[i].elapsed_time(r[i + 1]) for r in rec] for i in range(n_events - 1)]
 
     def entry(wname, shape, ms_lists, names, f_fwd, f_bwd, inputs):
-        e = {"shape": shape, "inputs": inputs, "steps": K, "warmup": Wm}
+        e = {"shape": shape, "inputs": inputs, "steps": K, "warmup": Wm,
+             "clocks": {k: last_clocks.get(k) for k in ("sm_mhz", "sm_mhz_min", "reasons", "samples")}}
         med = {n: statistics.median(v) for n, v in zip(names, ms_lists)}
         e["ms_median"] = {n: round(v, 4) for n, v in med.items()}
         e["fwd_tflops"] = round(f_fwd / med["fwd"] / 1e9, 1)
@@ -627,6 +643,8 @@ def other_configs(args, fa, torch, dev, stream, peak):
             e["bwd_pct_of_peak"] = round(100 * f_bwd / bwd_ms / 1e9 / peak, 2)
             e["bwd_main_tflops"] = round(f_bwd / med["bwd_main"] / 1e9, 1)
             e["bwd_main_frac"] = round(f_bwd / med["bwd_main"] / 1e9 / peak, 4)
+            e["bwd_main_frac_of_sustained"] = round(f_bwd / med["bwd_main"] / 1e9 / peak_sustained, 4)
+        e["fwd_frac_of_sustained"] = round(f_fwd / med["fwd"] / 1e9 / peak_sustained, 4)
         out[wname] = e
 
     def attn(wl, tensors, inputs, l2_flush):
@@ -704,7 +722,8 @@ def other_configs(args, fa, torch, dev, stream, peak):
     out["dec"] = {"shape": f"decode B={dw.B} Hq={dw.Hq} Hkv={dw.Hkv} Nq={dw.Nq} Nk={dw.Nk} d={dw.d} causal bf16",
                   "inputs": "seeded torch.randn on the device, iid N(0,1), rounded to bf16",
                   "ms_median": round(ms, 4), "gbs": round(algo / ms / 1e6, 1),
-                  "frac_of_hbm": round(algo / ms / 1e6 / float(peaks["hbm_gbs"]), 4), "steps": K, "warmup": Wm}
+                  "frac_of_hbm": round(algo / ms / 1e6 / float(peaks["hbm_gbs"]), 4), "steps": K, "warmup": Wm,
+                  "clocks": {k: last_clocks.get(k) for k in ("sm_mhz", "sm_mhz_min", "reasons", "samples")}}
     del flush
     return out
 

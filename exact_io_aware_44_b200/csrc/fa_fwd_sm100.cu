@@ -160,7 +160,8 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int u) {
 // The k-th unit of this CTA in a persistent grid of gridDim.x CTAs: rounds of
 // gridDim.x consecutive units, taken in snake order (CTA i takes the i-th unit of
 // even rounds and the i-th from the end of odd rounds), so that a CTA given a long
-// unit in one round gets a short one in the next. Returns n_units when done.
+// unit in one round gets a short one in the next. Returns n_units when done. (With
+// one CTA per unit the 0-th unit is blockIdx.x.)
 __device__ __forceinline__ int fwd_unit_index(int k, int n_units) {
   const int G = (int)gridDim.x;
   const int c = (int)blockIdx.x;
@@ -168,7 +169,9 @@ __device__ __forceinline__ int fwd_unit_index(int k, int n_units) {
   return u < n_units ? (int)u : n_units;
 }
 
-template <int D, int KIND>
+// PERSIST: the grid has fewer CTAs than units and every CTA loops over its share;
+// otherwise each CTA runs exactly one unit (blockIdx.x) and the unit loops fold away.
+template <int D, int KIND, bool PERSIST>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -242,7 +245,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         return true;
       };
       bool ok = true;
-      for (int k = 0; ok; ++k) {
+      for (int k = 0; ok && (PERSIST || k == 0); ++k) {
         const int u = fwd_unit_index(k, n_units);
         if (u >= n_units) break;
         const FwdUnit U = fwd_unit<C::kTiles>(p, u);
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     unsigned pv_count = 0;
     if (leader && prog) prog[blockIdx.x] = 0u;
     bool ok = true;
-    for (int k = 0; ok; ++k) {
+    for (int k = 0; ok && (PERSIST || k == 0); ++k) {
       const int u = fwd_unit_index(k, n_units);
       if (u >= n_units) break;
       const FwdUnit U = fwd_unit<C::kTiles>(p, u);
@@ -392,7 +395,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int s_base = 0;  // s_ready phases of this tile completed in earlier units
     int o_base = 0;  // o_done phases of this tile completed in earlier units
     bool ok = true;
-    for (int k = 0; ok; ++k) {
+    for (int k = 0; ok && (PERSIST || k == 0); ++k) {
       const int u = fwd_unit_index(k, n_units);
       if (u >= n_units) break;
       const FwdUnit U = fwd_unit<C::kTiles>(p, u);
@@ -556,9 +559,6 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          cudaStream_t stream) {
   using C = FwdCfg<D, KIND != kKindBf16>;
   static_assert(C::kSmemBytes <= 232448, "shared memory budget");
-  static std::atomic<uint64_t> configured{0};
-  cudaError_t e = ensure_smem_limit(fwd_kernel<D, KIND>, C::kSmemBytes, configured);
-  if (e != cudaSuccess) return e;
   // Short units (a few key tiles each) run persistently, one CTA per SM (the shared memory
   // and the 512 TMEM columns allow no more): the per-CTA set-up and ring fill would weigh on
   // every unit. Longer units get one CTA each, and the hardware's dynamic block scheduling
@@ -567,8 +567,18 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   const long long units = (long long)p.B * p.Hq * p.n_qblk;
   const int n_kv_all = (p.N + kTileN - 1) / kTileN;
   const int mean_kv = p.causal ? (n_kv_all + 1) / 2 : n_kv_all;  // key tiles of an average unit
-  const long long grid = mean_kv <= kPersistentMaxKv ? std::min<long long>(units, sm_count()) : units;
-  fwd_kernel<D, KIND><<<(unsigned)grid, kFwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  const bool persist = mean_kv <= kPersistentMaxKv && units > sm_count();
+  if (persist) {
+    static std::atomic<uint64_t> configured{0};
+    cudaError_t e = ensure_smem_limit(fwd_kernel<D, KIND, true>, C::kSmemBytes, configured);
+    if (e != cudaSuccess) return e;
+    fwd_kernel<D, KIND, true><<<(unsigned)sm_count(), kFwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  } else {
+    static std::atomic<uint64_t> configured{0};
+    cudaError_t e = ensure_smem_limit(fwd_kernel<D, KIND, false>, C::kSmemBytes, configured);
+    if (e != cudaSuccess) return e;
+    fwd_kernel<D, KIND, false><<<(unsigned)units, kFwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  }
   return cudaGetLastError();
 }
 
