@@ -912,7 +912,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c3",
-                    help="c2, c3, c3n, c5 (bf16 fwd+bwd), c4, c6 (bf16 fwd), f3, f4 (E4M3 fwd), f5 (E5M2 fwd), dec, dec4 (decode)")
+                    help="c2, c3, c3n, c5, c6b (bf16 fwd+bwd), c4, c6 (bf16 fwd), f3, f4 (E4M3 fwd), f5 (E5M2 fwd), dec, dec4 (decode)")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N>1: every rank runs the whole workload (weak scaling) or its slice of the heads (strong)")
     ap.add_argument("--e2e-steps", type=int, default=10)

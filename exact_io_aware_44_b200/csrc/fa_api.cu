@@ -428,7 +428,7 @@ int run_bwd(int phases, const void* q, const void* k, const void* v, const void*
   bool empty;
   int rc = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
   if (rc != FA_OK) return rc;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   if (empty) return FA_OK;
   const bool pre = phases & kPhasePre, main = phases & kPhaseMain, conv = phases & kPhaseConvert;
   if (!workspace) return FA_ERR_INVALID_ARG;

@@ -74,7 +74,7 @@ typedef enum {
  *   q [B,Hq,N,d] bf16, k/v [B,Hkv,N,d] bf16   inputs (read only)
  *   o [B,Hq,N,d] bf16                          output, round-to-nearest-even
  *   lse [B,Hq,N] float32                       output
- *   d must be 64, 128 or 256 (fa_bwd: 64 or 128). Arithmetic: bf16 operands, fp32
+ *   d must be 64, 128 or 256 (fa_bwd too). Arithmetic: bf16 operands, fp32
  *   accumulation; the probabilities P are rounded to bf16 before the P V product.
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -188,7 +188,8 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
  *   workspace         at least fa_bwd_workspace_bytes(...) bytes of device
  *                     memory, 256-byte aligned; its contents on entry do not matter.
  *                     It must not be used by another call in flight at the same time.
- *   d must be 64 or 128. dQ is accumulated with float32 atomics, so its last
+ *   d must be 64, 128 or 256 (d = 256 runs the query loop twice, once per half of
+ *   the head dim). dQ is accumulated with float32 atomics, so its last
  *   bits can vary from run to run; dK and dV are deterministic.
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,

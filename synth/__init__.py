@@ -24,6 +24,7 @@ Workloads (shapes from the pages' long-context regime; all synthetic, no dataset
   c5  bf16 fwd+bwd GQA, B=1 Hq=32 Hkv=8 N=32768 d=128, causal
   c3n bf16 fwd+bwd, c3's shape without the causal mask
   c6  bf16 fwd,  B=2 H=16 N=8192 d=256, causal
+  c6b bf16 fwd+bwd, c6's shape
   f3  E4M3 fwd,  B=2 H=32 N=8192 d=128, causal, std 1/sqrt(2) (c3's shape)
   f4  E4M3 fwd,  B=1 H=16 N=65536 d=128, causal (c4's shape)
   f5  E5M2 fwd,  c3's shape
@@ -102,6 +103,9 @@ WORKLOADS = {
     "c6": Workload("c6", 2, 16, 16, 8192, 256, True, "bf16", False, 1009,
                    std=1.0 / math.sqrt(2.0),
                    sample_heads=((0, 0), (0, 9), (1, 4), (1, 15)), sample_rows=256),
+    "c6b": Workload("c6b", 2, 16, 16, 8192, 256, True, "bf16", True, 1012,
+                    std=1.0 / math.sqrt(2.0),
+                    sample_heads=((0, 0), (0, 9), (1, 4), (1, 15)), sample_rows=256),
     "f3": Workload("f3", 2, 32, 32, 8192, 128, True, "e4m3", False, 1006,
                    std=1.0 / math.sqrt(2.0),
                    sample_heads=((0, 0), (0, 17), (1, 6), (1, 31)), sample_rows=256),

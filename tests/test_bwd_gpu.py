@@ -63,6 +63,24 @@ def test_bf16_bwd_small(cuda_device, shape, causal):
     check_full(w, cuda_device)
 
 
+D256_SHAPES = [
+    # B, Hq, Hkv, N (d = 256: 64-row query tiles, two passes over the head dim)
+    (1, 1, 1, 1),
+    (1, 2, 1, 65),
+    (1, 1, 1, 128),
+    (2, 2, 2, 300),
+    (1, 4, 2, 1000),
+]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("shape", D256_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_bf16_bwd_d256(cuda_device, shape, causal):
+    B, Hq, Hkv, N = shape
+    w = synth.small(B, Hq, Hkv, N, 256, causal, seed=950 + N)
+    check_full(w, cuda_device)
+
+
 def test_bf16_bwd_workspace_contents_do_not_matter(cuda_device):
     w = synth.small(1, 2, 1, 333, 128, True, seed=8)
     check_full(w, cuda_device, workspace_fill=float("nan"))
@@ -111,7 +129,7 @@ def sampled_bwd_check(w, device):
     return worst
 
 
-@pytest.mark.parametrize("name", ["c3", "c3n", "c5"])
+@pytest.mark.parametrize("name", ["c3", "c3n", "c5", "c6b"])
 def test_bf16_bwd_full_size_sampled(cuda_device, name):
     sampled_bwd_check(synth.WORKLOADS[name], cuda_device)
 
