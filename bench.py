@@ -586,9 +586,9 @@ def run_ours(args, w, world, rank, local):
 def other_configs(args, fa, torch, dev, stream, peak):
     """The remaining workloads the utilisation targets name, timed after the main
     line on the same device: the c4 forward, the c5 forward and backward, the c2
-    (d = 64) forward and backward, and one decode step. Same timing as the main
-    line: CUDA events around each launch on the launching stream, after warm-up,
-    no parity work inside. Inputs: c4, c5 and dec are drawn on the device by a
+    (d = 64) forward and backward, and two decode steps (dec, dec8). Same timing as
+    the main line: CUDA events around each launch on the launching stream, after
+    warm-up, no parity work inside. Inputs: c4, c5 and decode are drawn on the device by a
     seeded torch generator with the workloads' distributions (iid N(0, 1)), since
     they are larger than L2 and drawing them on the host would dominate the run;
     c2 uses the parity tests' seeded host recipe (with its spiked rows) and, being
@@ -695,35 +695,38 @@ def other_configs(args, fa, torch, dev, stream, peak):
     attn(wl, ts, "the parity tests' seeded host recipe (1% of query rows x20); L2 overwritten before each step",
          True)
     del ts
-    # decode: one new query per head against a 32768-key cache
-    dw = synth.DECODE_WORKLOADS["dec"]
-    gen.manual_seed(dw.seed)
-    qd = torch.randn((dw.B, dw.Hq, dw.Nq, dw.d), generator=gen, device=dev).to(torch.bfloat16)
-    kd = torch.randn((dw.B, dw.Hkv, dw.Nk, dw.d), generator=gen, device=dev).to(torch.bfloat16)
-    vd = torch.randn((dw.B, dw.Hkv, dw.Nk, dw.d), generator=gen, device=dev).to(torch.bfloat16)
-    od = torch.empty_like(qd)
-    ld = torch.empty((dw.B, dw.Hq, dw.Nq), dtype=torch.float32, device=dev)
-    wsd = torch.empty(fa.decode_workspace_bytes(dw.B, dw.Hq, dw.Hkv, dw.Nq, dw.Nk, dw.d), dtype=torch.uint8,
-                      device=dev)
+    # decode: one new query per head against a 32768-key cache (dec, 4 query rows a group), and
+    # eight new tokens per sequence of a 64-head model (dec8, 64 query rows a group)
+    for dname in ("dec", "dec8"):
+        dw = synth.DECODE_WORKLOADS[dname]
+        gen.manual_seed(dw.seed)
+        qd = torch.randn((dw.B, dw.Hq, dw.Nq, dw.d), generator=gen, device=dev).to(torch.bfloat16)
+        kd = torch.randn((dw.B, dw.Hkv, dw.Nk, dw.d), generator=gen, device=dev).to(torch.bfloat16)
+        vd = torch.randn((dw.B, dw.Hkv, dw.Nk, dw.d), generator=gen, device=dev).to(torch.bfloat16)
+        od = torch.empty_like(qd)
+        ld = torch.empty((dw.B, dw.Hq, dw.Nq), dtype=torch.float32, device=dev)
+        wsd = torch.empty(fa.decode_workspace_bytes(dw.B, dw.Hq, dw.Hkv, dw.Nq, dw.Nk, dw.d), dtype=torch.uint8,
+                          device=dev)
 
-    def dec_launch(evs):
-        if evs is not None:
-            evs[0].record(stream)
-        rc = fa.decode_raw(P(qd), P(kd), P(vd), P(od), P(ld), P(wsd), dw.B, dw.Hq, dw.Hkv, dw.Nq, dw.Nk, dw.d,
-                           dw.causal, dw.scale, 0, sp)
-        if rc:
-            raise fa.FAError(rc, "fa_decode")
-        if evs is not None:
-            evs[1].record(stream)
+        def dec_launch(evs):
+            if evs is not None:
+                evs[0].record(stream)
+            rc = fa.decode_raw(P(qd), P(kd), P(vd), P(od), P(ld), P(wsd), dw.B, dw.Hq, dw.Hkv, dw.Nq, dw.Nk, dw.d,
+                               dw.causal, dw.scale, 0, sp)
+            if rc:
+                raise fa.FAError(rc, "fa_decode")
+            if evs is not None:
+                evs[1].record(stream)
 
-    ms = statistics.median(timed(dec_launch, 2, False)[0])
-    peaks, _ = load_peaks()
-    algo = dw.kv_bytes() + 2 * qd.numel() * 2 + ld.numel() * 4
-    out["dec"] = {"shape": f"decode B={dw.B} Hq={dw.Hq} Hkv={dw.Hkv} Nq={dw.Nq} Nk={dw.Nk} d={dw.d} causal bf16",
-                  "inputs": "seeded torch.randn on the device, iid N(0,1), rounded to bf16",
-                  "ms_median": round(ms, 4), "gbs": round(algo / ms / 1e6, 1),
-                  "frac_of_hbm": round(algo / ms / 1e6 / float(peaks["hbm_gbs"]), 4), "steps": K, "warmup": Wm,
-                  "clocks": {k: last_clocks.get(k) for k in ("sm_mhz", "sm_mhz_min", "reasons", "samples")}}
+        ms = statistics.median(timed(dec_launch, 2, False)[0])
+        peaks, _ = load_peaks()
+        algo = dw.kv_bytes() + 2 * qd.numel() * 2 + ld.numel() * 4
+        out[dname] = {"shape": f"decode B={dw.B} Hq={dw.Hq} Hkv={dw.Hkv} Nq={dw.Nq} Nk={dw.Nk} d={dw.d} causal bf16",
+                      "inputs": "seeded torch.randn on the device, iid N(0,1), rounded to bf16",
+                      "ms_median": round(ms, 4), "gbs": round(algo / ms / 1e6, 1),
+                      "frac_of_hbm": round(algo / ms / 1e6 / float(peaks["hbm_gbs"]), 4), "steps": K, "warmup": Wm,
+                      "clocks": {k: last_clocks.get(k) for k in ("sm_mhz", "sm_mhz_min", "reasons", "samples")}}
+        del qd, kd, vd, od, ld, wsd
     del flush
     return out
 
@@ -849,7 +852,7 @@ def run_decode(args, w, world, rank, local):
                      "peak_source": f"{peak_src} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 2 * K,
+        "gpu_launches": 2 * K,  # the split kernel and the merge
         "clocks": clocks.summary(),
     }
 
@@ -912,7 +915,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c3",
-                    help="c2, c3, c3n, c5, c6b (bf16 fwd+bwd), c4, c6 (bf16 fwd), f3, f4 (E4M3 fwd), f5 (E5M2 fwd), dec, dec4 (decode)")
+                    help="c2, c3, c3n, c5, c6b (bf16 fwd+bwd), c4, c6 (bf16 fwd), f3, f4 (E4M3 fwd), f5 (E5M2 fwd), dec, dec4, dec8 (decode)")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N>1: every rank runs the whole workload (weak scaling) or its slice of the heads (strong)")
     ap.add_argument("--e2e-steps", type=int, default=10)

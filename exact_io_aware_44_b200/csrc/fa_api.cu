@@ -316,26 +316,34 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
 namespace fa {
 namespace {
 
-// Decode work split: all groups' 128-key chunks laid end to end and cut into
-// n_ctas equal slices, one per split-kernel CTA. Automatic: one CTA per SM of a
-// 148-SM part (the kernel keeps one CTA per SM), so the slices run as one wave;
-// num_splits > 0: B * Hkv * num_splits CTAs. Never more CTAs than chunks. A fixed
+// Decode work split. A GQA group's query rows ((Hq / Hkv) * Nq) are one unit when
+// they fit one CTA's MMA (at most 32 rows), else blocks of 128 rows, each a unit
+// of its own (row blocks). All units' 128-key chunks are laid end to end and cut
+// into n_ctas equal slices, one per split-kernel CTA. Automatic: one CTA per SM of
+// a 148-SM part (the kernels keep one CTA per SM), so the slices run as one wave;
+// num_splits > 0: units * num_splits CTAs. Never more CTAs than chunks. A fixed
 // rule of the sizes, not of the current device, so that the workspace size can be
-// computed without one. A slice may cross group boundaries; each (group, CTA)
-// piece is a segment with its own slot (group + CTA index) in the workspace.
+// computed without one. A slice may cross unit boundaries; each (unit, CTA) piece
+// is a segment with its own slot (unit + CTA index) in the workspace.
 constexpr int kDecodeSms = 148;
+constexpr int kDecodeBlockRows = 128;
 
 struct DecodeSplit {
-  int n_chunks, n_ctas;
+  int n_rb, slot_rows, n_chunks, n_ctas;
   long long total_chunks;
-  long long n_slots() const { return total_chunks / n_chunks + n_ctas - 1; }
+  long long n_units() const { return total_chunks / n_chunks; }
+  long long n_slots() const { return n_units() + n_ctas - 1; }
 };
 
-DecodeSplit decode_split(int B, int Hkv, int Nk, int num_splits) {
+DecodeSplit decode_split(int B, int Hq, int Hkv, int Nq, int Nk, int num_splits) {
+  const int rows = (Hq / Hkv) * Nq;
+  const int n_rb = rows <= 32 ? 1 : (rows + kDecodeBlockRows - 1) / kDecodeBlockRows;
+  const int slot_rows = n_rb == 1 ? rows : kDecodeBlockRows;
   const int n_chunks = (Nk + kTileN - 1) / kTileN;
-  const long long total = (long long)B * Hkv * n_chunks;
-  const long long want = num_splits > 0 ? (long long)B * Hkv * num_splits : kDecodeSms;
-  return {n_chunks, (int)std::min(want, total), total};
+  const long long units = (long long)B * Hkv * n_rb;
+  const long long total = units * n_chunks;
+  const long long want = num_splits > 0 ? units * num_splits : kDecodeSms;
+  return {n_rb, slot_rows, n_chunks, (int)std::min(want, total), total};
 }
 
 int check_decode(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale) {
@@ -344,15 +352,19 @@ int check_decode(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, floa
   if (rc != FA_OK) return rc;
   if (Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
   if (causal && Nq > Nk) return FA_ERR_INVALID_ARG;
-  if (d != 128 || (long long)(Hq / Hkv) * Nq > 32) return FA_ERR_UNSUPPORTED;
-  if ((long long)B * Hkv * (long long)Nk >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  const long long rows = (long long)(Hq / Hkv) * Nq;
+  const long long n_rb = rows <= 32 ? 1 : (rows + kDecodeBlockRows - 1) / kDecodeBlockRows;
+  if (rows >= (1ll << 31) || (long long)B * Hkv * n_rb * ((Nk + kTileN - 1) / kTileN) >= (1ll << 31) ||
+      (long long)B * Hkv * Nk >= (1ll << 31))
+    return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
-size_t decode_workspace(int B, int Hq, int Hkv, int Nq, int d, const DecodeSplit& sp) {
-  const size_t rows = (size_t)(Hq / Hkv) * Nq;  // query rows of a group
-  const size_t opart = ((size_t)sp.n_slots() * rows * d * sizeof(float) + 255) & ~size_t(255);
-  return opart + (size_t)sp.n_slots() * rows * sizeof(float);
+size_t decode_workspace(int d, const DecodeSplit& sp) {
+  const size_t slot_rows = (size_t)sp.slot_rows;
+  const size_t opart = ((size_t)sp.n_slots() * slot_rows * d * sizeof(float) + 255) & ~size_t(255);
+  return opart + (size_t)sp.n_slots() * slot_rows * sizeof(float);
 }
 
 }  // namespace
@@ -362,7 +374,7 @@ extern "C" {
 
 size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {
   if (check_decode(B, Hq, Hkv, Nq, Nk, d, 0, 1.f) != FA_OK) return 0;
-  return decode_workspace(B, Hq, Hkv, Nq, d, decode_split(B, Hkv, Nk, num_splits));
+  return decode_workspace(d, decode_split(B, Hq, Hkv, Nq, Nk, num_splits));
 }
 
 int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace, int B, int Hq,
@@ -374,7 +386,7 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_ALIGNMENT;
   DeviceInfo* di;
   if ((rc = current_device(&di)) != FA_OK) return rc;
-  const DecodeSplit sp = decode_split(B, Hkv, Nk, num_splits);
+  const DecodeSplit sp = decode_split(B, Hq, Hkv, Nq, Nk, num_splits);
   const long long rows = (long long)B * Hq * Nq;
   CUtensorMap tq, tk, tv;
   if ((rc = make_map(&tq, q, d, (int)rows, 1, decode_rows_per_cta((Hq / Hkv) * Nq))) != FA_OK) return rc;
@@ -385,7 +397,7 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.lse = lse;
   p.o_part = static_cast<float*>(workspace);
   const int g_rows = (Hq / Hkv) * Nq;
-  const size_t opart = ((size_t)sp.n_slots() * g_rows * d * sizeof(float) + 255) & ~size_t(255);
+  const size_t opart = ((size_t)sp.n_slots() * sp.slot_rows * d * sizeof(float) + 255) & ~size_t(255);
   p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + opart);
   p.status = di->status;
   p.B = B;
@@ -395,6 +407,8 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.Nk = Nk;
   p.causal = causal ? 1 : 0;
   p.rows = g_rows;
+  p.n_rb = sp.n_rb;
+  p.slot_rows = sp.slot_rows;
   p.n_chunks = sp.n_chunks;
   p.n_ctas = sp.n_ctas;
   p.total_chunks = sp.total_chunks;

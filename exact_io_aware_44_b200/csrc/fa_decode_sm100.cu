@@ -121,6 +121,20 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
+// One TMEM column (thread = lane).
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& v) {
+  asm volatile(
+      "{\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t"
+      "}"
+      : "=r"(v)
+      : "r"(taddr)
+      : "memory");
+}
 __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
@@ -463,6 +477,381 @@ __global__ void __launch_bounds__(DecCfg<R>::kThreads, 1)
   }
 }
 
+// Groups of more than 32 query rows: the query rows are the MMA's M, as in the
+// forward pass. A group's rows are cut into blocks of 128 (row blocks); each row
+// block is a unit of its own in the chunk sequence, so a group of more than 128
+// rows reads its keys once per row block.
+//   warp 0      TMA producer: the row block's 128 query rows (one buffer, released
+//               after the segment's last S), K and V chunks through a 3-stage ring.
+//   warp 1      allocates TMEM (512 columns); lane 0 issues
+//                 S(c) = Q K_c^T   M = 128 query rows, N = 128 keys, K = d -> S buffer c & 1
+//                 O   += P(c) V_c  A = P from TMEM (TS MMA), N = d            -> O buffer
+//               with S two chunks ahead of O and one O buffer per segment parity.
+//   warps 4-11  the forward pass's online softmax (reference max raised only when the
+//               row max grows by more than 2^8), thread = query row = TMEM lane; warps
+//               4-7 take keys [0,64) of every chunk and warps 8-11 keys [64,128), so two
+//               warps share each sub-partition (warps 2 and 3 only complete the first
+//               warpgroup, whose registers go to the softmax: 120 / 192 of 168 at
+//               launch). The two threads of a row exchange their maxima through shared
+//               memory every chunk (a thread writes the next chunk's only once p_full of
+//               this one is complete, i.e. after its partner has read it) and their
+//               shares of the denominator at a segment's end (through the S buffer's
+//               unused columns). P in bf16 over the first 64 columns of the S
+//               buffer; at a segment's end O / l and the LSE go to the segment's slot.
+//               Warps whose rows all lie past the group's end compute nothing and store
+//               P = 0.
+// TMEM columns: S buffers [0,128) and [128,256), O buffers [256,384) and [384,512).
+struct DecWideCfg {
+  static constexpr int D = 128;
+  static constexpr int kBlockRows = 128;
+  static constexpr int kThreads = 384;
+  static constexpr int kRegsLaunch = 168, kRegsControl = 120, kRegsSoftmax = 192;
+  static_assert(kThreads * kRegsLaunch == 128 * kRegsControl + 256 * kRegsSoftmax, "register split");
+  static constexpr int kKV = kDecChunk * D * 2;           // one K or V chunk (32 KB)
+  static constexpr int kRegion = kDecChunk * 128;         // 64-column block of a 128-row tile (16 KB)
+  static constexpr int kOffQ = 0;                         // one buffer x 2 blocks
+  static constexpr int kOffKV = kOffQ + 2 * kRegion;      // stages of K then V
+  static constexpr int kOffBar = kOffKV + kDecStages * 2 * kKV;
+  // q_full, q_empty, kv_full[3], kv_empty[3], s_full[2], p_full[2], pv_done[2], mma_done, xch
+  static constexpr int kNumBars = 16;
+  static constexpr int kOffRed = kOffBar + kNumBars * 8;  // [2][128] floats: row maxima by key half
+  static constexpr int kOffMisc = kOffRed + 2 * kBlockRows * 4;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static_assert(kOffKV % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static constexpr int kColS = 0, kColO = 256;
+};
+
+__global__ void __launch_bounds__(DecWideCfg::kThreads, 1)
+    decode_split_wide_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                             const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
+  using C = DecWideCfg;
+  constexpr int S = kDecStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024d(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;
+  uint64_t* kv_empty = bars + 5;
+  uint64_t* s_full = bars + 8;
+  uint64_t* p_full = bars + 10;
+  uint64_t* pv_done = bars + 12;
+  uint64_t* mma_done = bars + 14;
+  uint64_t* xch = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nch = p.n_chunks;  // chunks per row block
+  const long long f0 = (long long)blockIdx.x * p.total_chunks / p.n_ctas;
+  const long long f1 = (long long)(blockIdx.x + 1) * p.total_chunks / p.n_ctas;
+  const int n = (int)(f1 - f0);
+  const ChunkPos pos0{(int)(f0 / nch), (int)(f0 % nch), 0};  // G: row block (group * n_rb + block)
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 256);
+      mbar_init(&pv_done[b], 1);
+    }
+    mbar_init(xch, 256);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx w{abort_flag, p.status, p.wait_budget_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    regs_dec<C::kRegsControl, C::kRegsLaunch>();
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      bool ok = true;
+      int issued = 0, q_issued = 0;
+      ChunkPos ps = pos0;
+      for (int c = 0; c < n && ok; ++c, ps.next(nch)) {
+        const int grp = ps.G / p.n_rb;
+        if (c == 0 || ps.cig == 0) {
+          const int k = ps.seg;
+          if (!(ok = mbar_wait_spin(q_empty, (k & 1) ^ 1, w))) break;
+          ++q_issued;
+          mbar_arrive_expect_tx(q_full, 2 * C::kRegion);
+          const int row0 = grp * p.rows + (ps.G % p.n_rb) * C::kBlockRows;
+          for (int z = 0; z < 2; ++z) tma_load_3d(smem + C::kOffQ + z * C::kRegion, &tmQ, q_full, z * 64, row0, 0);
+        }
+        const int s = c % S;
+        if (!(ok = mbar_wait_spin(&kv_empty[s], ((c / S) & 1) ^ 1, w))) break;
+        ++issued;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * C::kKV);
+        const int key0 = ps.cig * kDecChunk;
+        uint8_t* st = smem + C::kOffKV + s * 2 * C::kKV;
+        for (int z = 0; z < 2; ++z) {
+          tma_load_3d(st + z * C::kRegion, &tmK, &kv_full[s], z * 64, key0, grp);
+          tma_load_3d(st + C::kKV + z * C::kRegion, &tmV, &kv_full[s], z * 64, key0, grp);
+        }
+      }
+      if (!ok) {
+        WaitCtx drain{abort_flag, p.status, 20000000ull};
+        volatile int zero = 0;
+        drain.abort_flag = &zero;
+        for (int c = max(0, issued - S); c < issued; ++c) mbar_wait(&kv_full[c % S], (c / S) & 1, drain);
+        if (q_issued > 0) mbar_wait(q_full, (q_issued - 1) & 1, drain);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    regs_dec<C::kRegsControl, C::kRegsLaunch>();
+    const bool leader = lane == 0;
+    constexpr uint32_t kIdS = idesc_bf16_f32(128, kDecChunk, false, false);  // S = Q K^T
+    constexpr uint32_t kIdO = idesc_bf16_f32(128, C::D, false, true);        // O += P V
+    const uint64_t d_q = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+    const uint64_t d_k = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);
+    const uint64_t d_v = sdesc_sw128(smem_u32(smem + C::kOffKV + C::kKV), C::kRegion, 1024);
+    // S(c) with the query rows of its segment; the Q buffer is released after the
+    // segment's last S
+    auto issue_s = [&](int c, const ChunkPos& ps) -> bool {
+      if (c == 0 || ps.cig == 0) {
+        if (!warp_wait_spin(q_full, ps.seg & 1, w)) return false;
+      }
+      if (!warp_wait_spin(&kv_full[c % S], (c / S) & 1, w)) return false;
+      tc_fence_after();
+      const uint64_t b0 = desc_advance(d_k, (c % S) * 2 * C::kKV);
+#pragma unroll
+      for (int k = 0; k < C::D / 16; ++k) {
+        const uint32_t off = (k >> 2) * C::kRegion + (k & 3) * 32;
+        if (leader)
+          mma_bf16_ss(tmem + C::kColS + (c & 1) * 128, desc_advance(d_q, off), desc_advance(b0, off), kIdS,
+                      k > 0 ? 1u : 0u);
+      }
+      if (leader) {
+        mma_commit(&s_full[c & 1]);
+        if (c == n - 1 || ps.cig == nch - 1) mma_commit(q_empty);
+      }
+      return true;
+    };
+    // O += P(c) V_c into the O buffer of its segment, overwriting at a segment's first chunk
+    auto issue_pv = [&](int c, const ChunkPos& pp) -> bool {
+      const uint64_t b0 = desc_advance(d_v, (c % S) * 2 * C::kKV);
+      const bool first = c == 0 || pp.cig == 0;
+      const uint32_t a = tmem + C::kColS + (c & 1) * 128;
+#pragma unroll
+      for (int k = 0; k < kDecChunk / 16; ++k) {
+        if (leader)
+          mma_bf16_ts(tmem + C::kColO + (pp.seg & 1) * 128, a + k * 8, desc_advance(b0, k * 16 * 128), kIdO,
+                      (!first || k > 0) ? 1u : 0u);
+      }
+      if (leader) {
+        mma_commit(&pv_done[c & 1]);
+        mma_commit(&kv_empty[c % S]);
+      }
+      return true;
+    };
+    bool ok = true;
+    ChunkPos ps = pos0, pp = pos0;  // ps runs two chunks ahead of pp
+    for (int c = 0; c < 2 && c < n && ok; ++c, ps.next(nch)) ok = issue_s(c, ps);
+    for (int c = 0; c < n && ok; ++c, pp.next(nch)) {
+      if (!(ok = warp_wait_spin(&p_full[c & 1], (c >> 1) & 1, w))) break;
+      tc_fence_after();
+      if (!(ok = issue_pv(c, pp))) break;
+      // S(c + 2) into the columns of P(c): the MMAs run in issue order, so P V(c) reads
+      // P(c) before S(c + 2) overwrites it
+      if (c + 2 < n) {
+        if (!(ok = issue_s(c + 2, ps))) break;
+        ps.next(nch);
+      }
+    }
+    if (leader) mma_commit(mma_done);
+    __syncwarp();
+    WaitCtx drain{abort_flag, p.status, 20000000ull};
+    volatile int zero = 0;
+    drain.abort_flag = &zero;
+    mbar_wait(mma_done, 0, drain);
+  } else if (warp < 4) {
+    regs_dec<C::kRegsControl, C::kRegsLaunch>();
+  } else {
+    // ------------------------------------------------------------ softmax (thread = query row)
+    regs_inc<C::kRegsSoftmax, C::kRegsLaunch>();
+    const int quarter = warp & 3;
+    const int h = (warp - 4) >> 2;      // key half of every chunk: [64h, 64h + 64)
+    const int r = quarter * 32 + lane;  // row of the block, TMEM lane
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float c2 = p.scale_log2;
+    // every valid row sees the keys up to all_vis
+    const int all_vis = p.causal ? p.Nk - p.Nq : p.Nk - 1;
+    float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+    float m_ref = -INFINITY;  // reference max, log2 units (S c)
+    float l = 0.f;            // this half's share of the denominator
+    int lim = -1;             // last key this row sees; -1 for rows past the group's end
+    bool dead = true;         // every row of this warp lies past the group's end
+    uint32_t xph = 0;
+    auto exchange = [&]() -> bool {  // all 256 softmax threads
+      mbar_arrive(xch);
+      const bool res = warp_wait(xch, xph, w);
+      xph ^= 1u;
+      return res;
+    };
+    bool ok = true;
+    ChunkPos pos = pos0;
+    for (int c = 0; c < n && ok; ++c, pos.next(nch)) {
+      const bool seg_first = c == 0 || pos.cig == 0;
+      const bool seg_last = c == n - 1 || pos.cig == nch - 1;
+      if (seg_first) {
+        const int j = (pos.G % p.n_rb) * C::kBlockRows + r;  // row of the group: query j mod Nq of its head
+        m_ref = -INFINITY;
+        l = 0.f;
+        lim = j >= p.rows ? -1 : (p.causal ? p.Nk - p.Nq + j % p.Nq : p.Nk - 1);
+        dead = __all_sync(0xffffffffu, lim < 0);
+      }
+      if (!(ok = warp_wait(&s_full[c & 1], (c >> 1) & 1, w))) break;
+      tc_fence_after();
+      const uint32_t tS = tmem + lane_off + C::kColS + (c & 1) * 128;
+      constexpr int kHalf = kDecChunk / 2;
+      float x[kHalf];
+      float mx = -INFINITY;
+      if (!dead) {
+#pragma unroll
+        for (int cc = 0; cc < kHalf / 32; ++cc) {
+          uint32_t rr[32];
+          tmem_ld32(tS + h * kHalf + cc * 32, rr);
+          tmem_ld_wait(rr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(rr[i]) * c2;
+        }
+        const int k0 = pos.cig * kDecChunk + h * kHalf;
+        if (k0 + kHalf - 1 > all_vis || lim < 0) {  // the causal edge, keys past Nk, rows past the end
+#pragma unroll
+          for (int i = 0; i < kHalf; ++i)
+            if (k0 + i > lim) x[i] = -INFINITY;
+        }
+        float mq[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+        for (int i = 4; i < kHalf; i += 8) {
+          mq[0] = fmax3(mq[0], x[i], x[i + 1]);
+          mq[1] = fmax3(mq[1], x[i + 2], x[i + 3]);
+          mq[2] = fmax3(mq[2], x[i + 4], x[i + 5]);
+          if (i + 6 < kHalf) mq[3] = fmax3(mq[3], x[i + 6], x[i + 7]);
+        }
+        mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
+      }
+      // the row max over the whole chunk: this half's and the partner's. The slot is written
+      // once p_full of the previous chunk is complete, i.e. once the partner has read it.
+      if (c > 0 && !(ok = warp_wait(&p_full[(c - 1) & 1], ((c - 1) >> 1) & 1, w))) break;
+      red[h * C::kBlockRows + r] = mx;
+      if (!(ok = exchange())) break;
+      const float m_new = fmaxf(m_ref, fmaxf(mx, red[(1 - h) * C::kBlockRows + r]));
+      float alpha = 1.f;
+      bool rescale = false;
+      if (m_new > m_ref + (float)kDecRescaleLog2) {
+        // O holds earlier chunks of this segment only if some of them had a visible key
+        if (!seg_first && m_ref != -INFINITY) {
+          alpha = ex2(m_ref - m_new);
+          l *= alpha;
+          rescale = true;
+        }
+        m_ref = m_new;
+      }
+      const float mc = m_ref == -INFINITY ? 0.f : m_ref;
+      uint32_t pk[kHalf / 2];
+      if (!dead) {
+        uint64_t rs2 = f2_pack(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < kHalf; i += 2) {
+          const float e0 = ex2(x[i] - mc), e1 = ex2(x[i + 1] - mc);
+          rs2 = f2_add(rs2, f2_pack(e0, e1));
+          pk[i / 2] = pack_bf16x2(e0, e1);
+        }
+        float ra, rb;
+        f2_unpack(rs2, ra, rb);
+        l += ra + rb;
+      } else {
+#pragma unroll
+        for (int i = 0; i < kHalf / 2; ++i) pk[i] = 0u;
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+        // this half's columns of the segment's O once P V(c - 1) is complete
+        if (!(ok = warp_wait(&pv_done[(c - 1) & 1], ((c - 1) >> 1) & 1, w))) break;
+        tc_fence_after();
+        const uint32_t tO = tmem + lane_off + C::kColO + (pos.seg & 1) * 128 + h * (C::D / 2);
+#pragma unroll
+        for (int cc = 0; cc < C::D / 64; ++cc) {
+          uint32_t rr[32];
+          tmem_ld32(tO + cc * 32, rr);
+          tmem_ld_wait(rr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+          tmem_st32(tO + cc * 32, rr);
+        }
+      }
+      float l_row = 0.f;
+      if (seg_last) {
+        // the row's denominator: both halves' shares, through column 64 + h of S(c), which
+        // both halves have read by now and P does not reach
+        tmem_st1(tS + kHalf + h, __float_as_uint(l));
+        tmem_st_wait();
+        tc_fence_before();
+        if (!(ok = exchange())) break;
+        tc_fence_after();
+        uint32_t other;
+        tmem_ld1(tS + kHalf + 1 - h, other);
+        l_row = l + __uint_as_float(other);
+      }
+      tmem_st32(tS + h * (kHalf / 2), pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[c & 1]);
+      if (seg_last && !dead) {
+        // end of a segment: this half's columns of O / l, and the LSE, into the segment's slot
+        if (!(ok = warp_wait(&pv_done[c & 1], (c >> 1) & 1, w))) break;
+        tc_fence_after();
+        const uint32_t tO = tmem + lane_off + C::kColO + (pos.seg & 1) * 128 + h * (C::D / 2);
+        const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+        const size_t slot_row = (size_t)(pos.G + (int)blockIdx.x) * p.slot_rows + r;
+        float4* dst = reinterpret_cast<float4*>(p.o_part + slot_row * C::D + h * (C::D / 2));
+#pragma unroll
+        for (int cc = 0; cc < C::D / 64; ++cc) {
+          uint32_t rr[32];
+          tmem_ld32(tO + cc * 32, rr);
+          tmem_ld_wait(rr);
+          if (lim >= 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              dst[(cc * 32 + i) / 4] = make_float4(__uint_as_float(rr[i]) * inv, __uint_as_float(rr[i + 1]) * inv,
+                                                   __uint_as_float(rr[i + 2]) * inv, __uint_as_float(rr[i + 3]) * inv);
+          }
+        }
+        if (h == 0 && lim >= 0)
+          p.lse_part[slot_row] = l_row > 0.f ? (m_ref + log2f(l_row)) * 0.6931471805599453f : -INFINITY;
+        tc_fence_before();  // the O reads, before a later segment's P V overwrites the buffer
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // The CTA whose slice of the chunk sequence holds chunk x: the largest i with
 // floor(i * total / n_ctas) <= x.
 __device__ __forceinline__ int decode_cta_of(long long x, const DecodeParams& p) {
@@ -479,15 +868,16 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock) decode_merge_kernel(c
   const long long row = (long long)blockIdx.x * kMergeRowsPerBlock + (threadIdx.x >> 5);
   if (row >= p.rows_total) return;
   const int lane = threadIdx.x & 31;
-  const int G = (int)(row / p.rows);
-  const int q = (int)(row % p.rows);
+  const int q = (int)(row % p.rows);                                // row of its group
+  const int G = (int)(row / p.rows) * p.n_rb + q / p.slot_rows;     // its row block's unit
+  const int sq = q % p.slot_rows;                                   // row within the slot
   const int i0 = decode_cta_of((long long)G * p.n_chunks, p);
   const int i1 = decode_cta_of((long long)(G + 1) * p.n_chunks - 1, p);
   float m = -INFINITY, wsum = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
   for (int i = i0; i <= i1; ++i) {
-    const size_t slot_row = (size_t)(G + i) * p.rows + q;
+    const size_t slot_row = (size_t)(G + i) * p.slot_rows + sq;
     const float ls = p.lse_part[slot_row];
     const float4 o4 = reinterpret_cast<const float4*>(p.o_part + slot_row * 128)[lane];
     if (ls == -INFINITY) continue;  // no visible key in this segment
@@ -528,12 +918,29 @@ cudaError_t launch_decode_r(const CUtensorMap& tq, const CUtensorMap& tk, const 
   return cudaGetLastError();
 }
 
-int decode_rows_per_cta(int rows) { return rows <= 16 ? 16 : 32; }
+cudaError_t launch_decode_wide(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const DecodeParams& p, cudaStream_t s) {
+  using C = DecWideCfg;
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = ensure_smem_limit(decode_split_wide_kernel, C::kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
+  decode_split_wide_kernel<<<(unsigned)p.n_ctas, C::kThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_merge_kernel<<<(unsigned)((p.rows_total + kMergeRowsPerBlock - 1) / kMergeRowsPerBlock),
+                        32 * kMergeRowsPerBlock, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+int decode_rows_per_cta(int rows) { return rows <= 16 ? 16 : rows <= 32 ? 32 : DecWideCfg::kBlockRows; }
 
 cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           cudaStream_t s) {
-  return decode_rows_per_cta(p.rows) == 16 ? launch_decode_r<16>(tq, tk, tv, p, s)
-                                           : launch_decode_r<32>(tq, tk, tv, p, s);
+  switch (decode_rows_per_cta(p.rows)) {
+    case 16: return launch_decode_r<16>(tq, tk, tv, p, s);
+    case 32: return launch_decode_r<32>(tq, tk, tv, p, s);
+    default: return launch_decode_wide(tq, tk, tv, p, s);
+  }
 }
 
 }  // namespace fa

@@ -57,15 +57,17 @@ struct BwdParams {
 struct DecodeParams {
   void* o;            // bf16 [B, Hq, Nq, d]
   float* lse;         // [B, Hq, Nq]
-  float* o_part;      // workspace: per segment slot, normalised partial O [n_slots, rows, d]
-  float* lse_part;    // workspace: per segment slot, partial LSE (natural log) [n_slots, rows]
+  float* o_part;      // workspace: per segment slot, normalised partial O [n_slots, slot_rows, d]
+  float* lse_part;    // workspace: per segment slot, partial LSE (natural log) [n_slots, slot_rows]
   int* status;
   int B, Hq, Hkv, Nq, Nk;
   int causal;
   int rows;                        // query rows of a GQA group: (Hq / Hkv) * Nq
-  int n_chunks;                    // 128-key chunks per group
-  int n_ctas;                      // split-kernel CTAs (equal slices of all groups' chunks)
-  long long total_chunks;          // B * Hkv * n_chunks
+  int n_rb;                        // row blocks per group (units of the chunk sequence)
+  int slot_rows;                   // query rows of a workspace slot (of a row block)
+  int n_chunks;                    // 128-key chunks per row block
+  int n_ctas;                      // split-kernel CTAs (equal slices of all row blocks' chunks)
+  long long total_chunks;          // B * Hkv * n_rb * n_chunks
   long long rows_total;            // B * Hq * Nq
   float scale_log2;
   uint64_t wait_budget_ns;
@@ -82,7 +84,8 @@ cudaError_t launch_fwd_e5m2(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const FwdParams& p, cudaStream_t s);
 cudaError_t launch_fwd_f32(const FwdF32Params& p, cudaStream_t s);
 // Decode: the split kernel, then the merge of the splits.
-// Query rows per decode CTA for a GQA group of `rows` rows (16 or 32).
+// Query rows per decode CTA for a GQA group of `rows` rows: 16 or 32 (one CTA's
+// MMA N covers the group), else 128 (a row block, the MMA M).
 int decode_rows_per_cta(int rows);
 cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           cudaStream_t s);

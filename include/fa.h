@@ -116,12 +116,16 @@ int fa_fwd_e5m2(const void* q, const void* k, const void* v, float descale_q, fl
 /*
  * fa_decode_workspace_bytes -- device scratch that fa_decode needs.
  *
- * The split kernel cuts all (batch, kv head) groups' 128-key chunks, laid end to
- * end, into n_ctas equal slices; each piece of a slice inside one group has a
- * slot holding a float32 partial output [rows, d] and partial LSE [rows], with
- * rows = (Hq / Hkv) * Nq, and there are B*Hkv + n_ctas - 1 slots. n_ctas is 148
+ * A (batch, kv head) group has rows = (Hq / Hkv) * Nq query rows. Up to 32 rows
+ * the group is one unit; above that its rows are cut into n_rb = ceil(rows / 128)
+ * row blocks, each a unit of its own. The split kernel cuts all units' 128-key
+ * chunks, laid end to end, into n_ctas equal slices; each piece of a slice inside
+ * one unit has a slot holding a float32 partial output [slot_rows, d] and partial
+ * LSE [slot_rows], where slot_rows = rows for n_rb = 1 and 128 otherwise; there
+ * are units + n_ctas - 1 slots, units = B*Hkv*n_rb. The workspace holds all slots'
+ * outputs (padded to a multiple of 256 bytes), then all their LSEs. n_ctas is 148
  * for num_splits <= 0 (a fixed rule of the sizes, so no device is needed here),
- * else B*Hkv*num_splits, and never more than the chunks. Returns 0 for sizes
+ * else units*num_splits, and never more than the chunks. Returns 0 for sizes
  * fa_decode rejects.
  */
 size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits);
@@ -137,18 +141,21 @@ size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, 
  * j <= Nk - Nq + i (Nq = Nk gives fa_fwd's square causal mask). Each key split
  * computes a partial softmax over its keys; the partials are combined with the
  * online-softmax merge (running max, rescaled denominators: the update of the
- * card's first paragraph), LSE = log sum_s e^(LSE_s), O = sum_s e^(LSE_s - LSE) O_s.
+ * card's first paragraph), LSE = log sum_s e^(LSE_s), O = sum_s e^(LSE_s - LSE) O_s,
+ * by a second kernel (one warp per query row).
  *   q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] bf16   inputs (read only)
  *   o [B,Hq,Nq,d] bf16, lse [B,Hq,Nq] float32   outputs, as in fa_fwd
  *   workspace   at least fa_decode_workspace_bytes(..., num_splits) bytes of
  *               device memory, 256-byte aligned, contents on entry irrelevant
  *   num_splits  work split: <= 0 gives one CTA per SM of a 148-SM part; > 0 gives
- *               B*Hkv*num_splits CTAs (about num_splits key splits per group); never
- *               more CTAs than 128-key chunks
- *   d must be 128 and (Hq / Hkv) * Nq at most 32 (one CTA serves a whole GQA
- *   group's query rows), else FA_ERR_UNSUPPORTED; causal with Nq > Nk is
- *   FA_ERR_INVALID_ARG. Arithmetic: bf16 operands, fp32 accumulation; P is
- *   rounded to bf16 before the P V product; the partials stay fp32.
+ *               units*num_splits CTAs (about num_splits key splits per group, or
+ *               per row block of 128 rows); never more CTAs than 128-key chunks
+ *   d must be 128, else FA_ERR_UNSUPPORTED; causal with Nq > Nk is
+ *   FA_ERR_INVALID_ARG. A group of up to 32 query rows is served by one CTA at a
+ *   time with the rows as the MMA's N, so its keys are read once; larger groups
+ *   take 128-row blocks as the MMA's M, and their keys are read once per block.
+ *   Arithmetic: bf16 operands, fp32 accumulation; P is rounded to bf16 before
+ *   the P V product; the partials stay fp32.
  */
 int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
               int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale, int num_splits,

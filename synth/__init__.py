@@ -29,6 +29,8 @@ Workloads (shapes from the pages' long-context regime; all synthetic, no dataset
   f4  E4M3 fwd,  B=1 H=16 N=65536 d=128, causal (c4's shape)
   f5  E5M2 fwd,  c3's shape
   dec decode,    B=16 Hq=32 Hkv=8, Nq=1 new query against Nk=32768 cached keys, d=128
+  dec4 decode,   B=16 Hq=32 Hkv=4, Nq=4 (32 query rows a group)
+  dec8 decode,   B=16 Hq=64 Hkv=8, Nq=8 (64 query rows a group)
 """
 from __future__ import annotations
 
@@ -261,6 +263,9 @@ DECODE_WORKLOADS = {
     "dec": DecodeWorkload("dec", 16, 32, 8, 1, 32768, 128, True, 1010),
     # speculative / multi-token decode: 4 new tokens per sequence, GQA group 8 (32 query rows a CTA)
     "dec4": DecodeWorkload("dec4", 16, 32, 4, 4, 32768, 128, True, 1011),
+    # 8 new tokens per sequence, 64 query heads over 8 kv heads: 64 query rows a group,
+    # the 128-row-block kernel
+    "dec8": DecodeWorkload("dec8", 16, 64, 8, 8, 32768, 128, True, 1013),
 }
 
 

@@ -87,9 +87,9 @@ def _dec(B=1, Hq=8, Hkv=1, Nq=1, Nk=1000, d=128, causal=1, scale=0.088, splits=0
 
 def test_decode_rejects_bad_arguments_on_host():
     assert _dec(d=64) == -2                        # d = 128 only
-    assert _dec(Hq=64, Hkv=1) == -2                # 64 query rows per group > 32
-    assert _dec(Hq=8, Nq=5) == -2                  # 40 rows > 32
-    assert _dec(Hq=16, Nq=3) == -2                 # 48 rows > 32
+    assert _dec(Hq=64, Hkv=1, ptr=0x1008) == -3    # 64 query rows per group: accepted up to the pointer check
+    assert _dec(Hq=8, Nq=5, ws=0x1010) == -3       # 40 rows: row blocks, past the size checks
+    assert _dec(Hq=16, Nq=3000, Nk=3000, ptr=0x1008) == -3   # 48000 rows: 375 row blocks
     assert _dec(Nq=5, Nk=4) == -1                  # causal needs Nq <= Nk
     assert _dec(Nk=0) == -1
     assert _dec(Hq=6, Hkv=4) == -1
@@ -99,27 +99,34 @@ def test_decode_rejects_bad_arguments_on_host():
     assert _dec(ws=0) == -1
 
 
-def _decode_slots(B, Hq, Hkv, Nq, Nk, splits):
-    """The work split restated: all groups' 128-key chunks end to end, cut into
-    n_ctas equal slices (one per SM of a 148-SM part, or B * Hkv * num_splits;
-    never more than the chunks); one workspace slot per (group, CTA) pair that
-    can meet, i.e. groups + n_ctas - 1."""
+def _decode_split(B, Hq, Hkv, Nq, Nk, splits):
+    """The work split restated: a group of up to 32 query rows is one unit, a larger
+    one is ceil(rows / 128) row blocks of 128; all units' 128-key chunks end to end,
+    cut into n_ctas equal slices (one per SM of a 148-SM part, or units * num_splits;
+    never more than the chunks); one workspace slot per (unit, CTA) pair that can
+    meet, i.e. units + n_ctas - 1, each of slot_rows rows."""
+    rows = Hq // Hkv * Nq
+    n_rb = 1 if rows <= 32 else -(-rows // 128)
+    slot_rows = rows if n_rb == 1 else 128
     n_chunks = -(-Nk // 128)
-    total = B * Hkv * n_chunks
-    n_ctas = min(B * Hkv * splits if splits > 0 else 148, total)
-    return B * Hkv + n_ctas - 1
+    units = B * Hkv * n_rb
+    n_ctas = min(units * splits if splits > 0 else 148, units * n_chunks)
+    return units + n_ctas - 1, slot_rows, units
 
 
 def test_decode_workspace_and_split_rule():
-    """Per slot: fp32 partial O (256-byte padded) and fp32 partial LSE per query row of a group."""
+    """Per slot: fp32 partial O (256-byte padded as a whole) and fp32 partial LSE per
+    query row of a slot."""
     d = 128
-    for (B, Hq, Hkv, Nq) in ((4, 32, 8, 1), (16, 32, 8, 1), (16, 32, 4, 4), (1, 8, 1, 3), (64, 16, 8, 1)):
+    for (B, Hq, Hkv, Nq) in ((4, 32, 8, 1), (16, 32, 8, 1), (16, 32, 4, 4), (1, 8, 1, 3), (64, 16, 8, 1),
+                             (16, 64, 1, 1), (2, 8, 1, 5), (16, 32, 2, 8), (1, 16, 1, 17), (3, 4, 1, 100)):
         for Nk, splits in ((128, 1), (4096, 4), (4096, 7), (100000, 0), (32768, 0), (777, 0), (1, 0), (200, 0)):
+            if Nq > Nk:
+                continue
             ws = fa.decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, splits)
-            slots = _decode_slots(B, Hq, Hkv, Nq, Nk, splits)
-            rows = Hq // Hkv * Nq
-            opart = (slots * rows * d * 4 + 255) // 256 * 256
-            assert ws == opart + slots * rows * 4, (B, Hq, Hkv, Nq, Nk, splits, ws)
+            slots, slot_rows, units = _decode_split(B, Hq, Hkv, Nq, Nk, splits)
+            pad = lambda x: (x + 255) // 256 * 256
+            assert ws == pad(slots * slot_rows * d * 4) + slots * slot_rows * 4, (B, Hq, Hkv, Nq, Nk, splits, ws)
     assert fa.decode_workspace_bytes(1, 8, 1, 1, 1000, 64, 0) == 0
 
 

@@ -53,6 +53,15 @@ SHAPES = [
     (1, 32, 4, 4, 9000),    # the same with 32 rows
     (64, 16, 8, 1, 200),    # 1024 chunks of short caches: about 4 segments per CTA
     (32, 32, 4, 3, 300),    # 24 rows, 3 chunks a group, segments across groups
+    # more than 32 rows a group: 128-row blocks with the rows as the MMA's M
+    (1, 8, 1, 5, 900),      # 40 rows, one block, 88 rows unused
+    (2, 64, 1, 1, 3000),    # a 64-head group (MQA)
+    (1, 16, 2, 8, 1000),    # GQA group 8 x 8 new tokens = 64 rows, the causal edge spans 8 keys
+    (2, 32, 2, 8, 2500),    # 128 rows: one full block
+    (1, 16, 1, 9, 700),     # 144 rows: a full block and a block of 16
+    (1, 4, 1, 100, 640),    # 400 rows: four blocks, the causal edge spans 100 keys
+    (1, 1, 1, 200, 200),    # square, 200 rows
+    (8, 32, 4, 5, 3000),    # 40 rows, 24 chunks a block over 148 CTAs: segments across blocks
 ]
 
 
@@ -113,7 +122,29 @@ def test_decode_repeatable_and_bounded_writes(cuda_device):
     assert torch.equal(o_buf[:n_o].view_as(q), o2) and torch.equal(l_buf[:16].view(2, 8, 1), l2)
 
 
-@pytest.mark.parametrize("name", ["dec", "dec4"])
+@pytest.mark.parametrize("shape", [(3, 8, 2, 1, 7000), (1, 16, 1, 9, 700), (2, 32, 4, 4, 2500)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_decode_workspace_reused_with_garbage(cuda_device, shape):
+    """One workspace, filled with garbage and reused across calls and split counts:
+    nothing in it carries over, so each result equals the oracle."""
+    import torch
+    import exact_io_aware_44_b200 as fa
+    B, Hq, Hkv, Nq, Nk = shape
+    w = synth.DecodeWorkload("ws" + "x".join(map(str, shape)), B, Hq, Hkv, Nq, Nk, 128, True, 3000 + Nk)
+    q, k, v = synth.decode_inputs(w)
+    dev = lambda x: to_dev(x, torch.bfloat16, cuda_device)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    nbytes = max(fa.decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, 128, s) for s in (0, 3, 7))
+    ws = torch.full((nbytes,), 0xFF, dtype=torch.uint8, device=cuda_device)
+    o_ref, lse_ref = oracle.decode_fwd64(q, k, v, True, w.scale)
+    for splits in (0, 7, 3, 0):
+        o, lse = fa.decode(qd, kd, vd, causal=True, num_splits=splits, workspace=ws)
+        assert fa.get_status() == 0
+        assert_fwd_ok(fwd_errors(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref),
+                      f"reused workspace splits={splits}")
+
+
+@pytest.mark.parametrize("name", ["dec", "dec4", "dec8"])
 def test_decode_full_size_workload(cuda_device, name):
     """The benchmark's decode steps (B=16 Hq=32 against 32768 cached keys: Hkv=8 with
     one new query, Hkv=4 with four), in the launch configuration the benchmark
@@ -122,7 +153,7 @@ def test_decode_full_size_workload(cuda_device, name):
     w = synth.DECODE_WORKLOADS[name]
     q, k, v, o, lse = run_decode(w, cuda_device)
     assert np.isfinite(o).all() and np.isfinite(lse).all()
-    for (b, h) in ((0, 0), (3, 9), (7, 31), (15, 16)):
+    for (b, h) in ((0, 0), (3, 9), (7, 31), (15, 16), (15, w.Hq - 1)):
         kvh = h // w.group
         o_ref, lse_ref = oracle.decode_fwd64(q[b:b + 1, h:h + 1], k[b:b + 1, kvh:kvh + 1], v[b:b + 1, kvh:kvh + 1],
                                              w.causal, w.scale)
