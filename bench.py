@@ -47,15 +47,16 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 # source makes the figure stale and the bench reports null.
 NCU_TRAFFIC = {
     # profiles/bwd_main_d128_B2H32N8192_causal.md
-    ("bwd_main", "c3"): {"bytes_per_launch": 810287616 + 489886208, "csrc_sha": "1896da15478db7ec"},
-    # profiles/bwd_main_d64_B4H16N2048_causal.md (--set full capture)
-    ("bwd_main", "c2"): {"bytes_per_launch": 101763584 + 22738176, "csrc_sha": "56c56e7e3931d08b"},
+    ("bwd_main", "c3"): {"bytes_per_launch": 810053376 + 491489280, "csrc_sha": "eca1cf4d70f597f7"},
+    # profiles/bwd_main_d64_B4H16N2048_causal.md
+    ("bwd_main", "c2"): {"bytes_per_launch": 101785600 + 24538112, "csrc_sha": "e795a43c1c31fa93"},
     # profiles/fwd_bf16_d128_B2H32N8192_causal.md
-    ("fwd", "c3"): {"bytes_per_launch": 404763136 + 118222336, "csrc_sha": "6850015faac09dea"},
-    ("fwd", "c4"): {"bytes_per_launch": 810670592 + 261153792, "csrc_sha": "6850015faac09dea"},
-    # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md
-    ("decode_split", "dec"): {"bytes_per_launch": 2148272896 + 3852544, "csrc_sha": "4137ec07188f1845"},
-    ("decode_split", "dec4"): {"bytes_per_launch": 1074823168 + 4116480, "csrc_sha": "4137ec07188f1845"},
+    ("fwd", "c3"): {"bytes_per_launch": 403261696 + 118636032, "csrc_sha": "3b3769599fbeb05b"},
+    ("fwd", "c4"): {"bytes_per_launch": 811248896 + 262354432, "csrc_sha": "3b3769599fbeb05b"},
+    # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md, profiles/decode_wide_B16Hq64Hkv8Nq8_Nk32768_d128.md
+    ("decode_split", "dec"): {"bytes_per_launch": 2148271104 + 3724800, "csrc_sha": "0bd30d5eb481de28"},
+    ("decode_split", "dec4"): {"bytes_per_launch": 1074862848 + 4931584, "csrc_sha": "0bd30d5eb481de28"},
+    ("decode_split", "dec8"): {"bytes_per_launch": 2153814528 + 8017408, "csrc_sha": "0bd30d5eb481de28"},
 }
 
 
