@@ -28,6 +28,10 @@
  *             must be 16-byte aligned. Outputs must not alias inputs.
  *   Streams   `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
  *             asynchronous: they enqueue work and return before it completes.
+ *             They neither allocate nor synchronise, so fa_fwd, fa_bwd and
+ *             fa_decode can be captured in a CUDA graph once one eager call on
+ *             the device has loaded the kernels (fa_get_status synchronises and
+ *             stays outside a capture).
  *   Errors    A negative return code means nothing was launched and no output
  *             was touched. FA_OK means the work was enqueued. A failure found on
  *             the device is recorded in a device status word; fa_get_status()
