@@ -6,14 +6,16 @@
 // ("FlashAttention Kernel & Online Softmax" card: the relation to the KV cache
 // and the decode bandwidth bottleneck). So the design goal is to read K and V
 // exactly once at full bandwidth. A GQA group (one batch entry and kv head: g
-// query heads x Nq queries, at most 32 rows) is the unit that shares K and V; its
-// keys form n_chunks chunks of 128. All groups' chunks are laid end to end, and
-// CTA i of the persistent grid (one CTA per SM) takes the i-th of n_ctas equal
-// slices of that sequence. A slice may cross group boundaries: each piece of it
-// that lies in one group is a segment, with its own partial output O_s and
-// log-sum-exp LSE_s, stored in slot (group + i) of the workspace. The key ring
+// query heads x Nq queries) of up to 32 rows is the unit that shares K and V
+// (decode_split_kernel<R>); a larger group is cut into 128-row blocks, each a unit
+// (decode_split_wide_kernel, below). A unit's keys form n_chunks chunks of 128.
+// All units' chunks are laid end to end, and CTA i of the persistent grid (one CTA
+// per SM) takes the i-th of n_ctas equal slices of that sequence. A slice may
+// cross unit boundaries: each piece of it that lies in one unit is a segment, with
+// its own partial output O_s and log-sum-exp LSE_s, stored in slot (unit + i) of
+// the workspace. The key ring
 // keeps streaming across segments, so an SM never waits for a new CTA to fill it.
-// decode_merge_kernel combines a group's segments with the online-softmax merge
+// decode_merge_kernel combines a unit's segments with the online-softmax merge
 // (running max and rescaled denominators, the same update the pages give for key
 // blocks): LSE = log sum_s e^(LSE_s), O = sum_s e^(LSE_s - LSE) O_s.
 //
