@@ -212,9 +212,9 @@ def decode_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, ws_ptr, B, Hq, Hkv, Nq, Nk, 
 def decode(q, k, v, causal: bool = True, scale: float | None = None, num_splits: int = 0, out=None, lse=None,
            workspace=None, stream=None):
     """Attention of q [B, Hq, Nq, d] (the last Nq positions) against a key/value
-    cache k, v [B, Hkv, Nk, d], all bf16, split along the keys; d = 128. A GQA
-    group's (Hq / Hkv) * Nq query rows form one unit up to 32 rows, else blocks of
-    128 rows. num_splits = 0: one CTA per SM, each an equal slice of all units'
+    cache k, v [B, Hkv, Nk, d], all bf16, split along the keys; d = 64 or 128. At
+    d = 128 a GQA group's (Hq / Hkv) * Nq query rows form one unit up to 32 rows,
+    else blocks of 128 rows (always at d = 64). num_splits = 0: one CTA per SM, each an equal slice of all units'
     128-key chunks; > 0: units * num_splits CTAs. Returns (o, lse)."""
     import torch
     if q.dim() != 4 or k.dim() != 4:

@@ -352,7 +352,7 @@ int check_decode(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, floa
   if (rc != FA_OK) return rc;
   if (Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
   if (causal && Nq > Nk) return FA_ERR_INVALID_ARG;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const long long rows = (long long)(Hq / Hkv) * Nq;
   const long long n_rb = rows <= 32 ? 1 : (rows + kDecodeBlockRows - 1) / kDecodeBlockRows;
   if (rows >= (1ll << 31) || (long long)B * Hkv * n_rb * ((Nk + kTileN - 1) / kTileN) >= (1ll << 31) ||
@@ -389,7 +389,7 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   const DecodeSplit sp = decode_split(B, Hq, Hkv, Nq, Nk, num_splits);
   const long long rows = (long long)B * Hq * Nq;
   CUtensorMap tq, tk, tv;
-  if ((rc = make_map(&tq, q, d, (int)rows, 1, decode_rows_per_cta((Hq / Hkv) * Nq))) != FA_OK) return rc;
+  if ((rc = make_map(&tq, q, d, (int)rows, 1, decode_rows_per_cta((Hq / Hkv) * Nq, d))) != FA_OK) return rc;
   if ((rc = make_map(&tk, k, d, Nk, B * Hkv)) != FA_OK) return rc;
   if ((rc = make_map(&tv, v, d, Nk, B * Hkv)) != FA_OK) return rc;
   DecodeParams p;
@@ -405,6 +405,7 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.Hkv = Hkv;
   p.Nq = Nq;
   p.Nk = Nk;
+  p.d = d;
   p.causal = causal ? 1 : 0;
   p.rows = g_rows;
   p.n_rb = sp.n_rb;

@@ -503,16 +503,18 @@ __global__ void __launch_bounds__(DecCfg<R>::kThreads, 1)
 //               Warps whose rows all lie past the group's end compute nothing and store
 //               P = 0.
 // TMEM columns: S buffers [0,128) and [128,256), O buffers [256,384) and [384,512).
+template <int D_>
 struct DecWideCfg {
-  static constexpr int D = 128;
+  static constexpr int D = D_;                             // head dim: 64 or 128
+  static constexpr int kRegions = D * 2 / 128;             // 64-column blocks of a row
   static constexpr int kBlockRows = 128;
   static constexpr int kThreads = 384;
   static constexpr int kRegsLaunch = 168, kRegsControl = 120, kRegsSoftmax = 192;
   static_assert(kThreads * kRegsLaunch == 128 * kRegsControl + 256 * kRegsSoftmax, "register split");
-  static constexpr int kKV = kDecChunk * D * 2;           // one K or V chunk (32 KB)
+  static constexpr int kKV = kDecChunk * D * 2;           // one K or V chunk (16 or 32 KB)
   static constexpr int kRegion = kDecChunk * 128;         // 64-column block of a 128-row tile (16 KB)
-  static constexpr int kOffQ = 0;                         // one buffer x 2 blocks
-  static constexpr int kOffKV = kOffQ + 2 * kRegion;      // stages of K then V
+  static constexpr int kOffQ = 0;                         // one buffer of kRegions blocks
+  static constexpr int kOffKV = kOffQ + kRegions * kRegion;  // stages of K then V
   static constexpr int kOffBar = kOffKV + kDecStages * 2 * kKV;
   // q_full, q_empty, kv_full[3], kv_empty[3], s_full[2], p_full[2], pv_done[2], mma_done, xch
   static constexpr int kNumBars = 16;
@@ -524,10 +526,11 @@ struct DecWideCfg {
   static constexpr int kColS = 0, kColO = 256;
 };
 
-__global__ void __launch_bounds__(DecWideCfg::kThreads, 1)
+template <int D>
+__global__ void __launch_bounds__(DecWideCfg<D>::kThreads, 1)
     decode_split_wide_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                              const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
-  using C = DecWideCfg;
+  using C = DecWideCfg<D>;
   constexpr int S = kDecStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024d(smem_raw);
@@ -595,9 +598,10 @@ __global__ void __launch_bounds__(DecWideCfg::kThreads, 1)
           const int k = ps.seg;
           if (!(ok = mbar_wait_spin(q_empty, (k & 1) ^ 1, w))) break;
           ++q_issued;
-          mbar_arrive_expect_tx(q_full, 2 * C::kRegion);
+          mbar_arrive_expect_tx(q_full, C::kRegions * C::kRegion);
           const int row0 = grp * p.rows + (ps.G % p.n_rb) * C::kBlockRows;
-          for (int z = 0; z < 2; ++z) tma_load_3d(smem + C::kOffQ + z * C::kRegion, &tmQ, q_full, z * 64, row0, 0);
+          for (int z = 0; z < C::kRegions; ++z)
+            tma_load_3d(smem + C::kOffQ + z * C::kRegion, &tmQ, q_full, z * 64, row0, 0);
         }
         const int s = c % S;
         if (!(ok = mbar_wait_spin(&kv_empty[s], ((c / S) & 1) ^ 1, w))) break;
@@ -605,7 +609,7 @@ __global__ void __launch_bounds__(DecWideCfg::kThreads, 1)
         mbar_arrive_expect_tx(&kv_full[s], 2 * C::kKV);
         const int key0 = ps.cig * kDecChunk;
         uint8_t* st = smem + C::kOffKV + s * 2 * C::kKV;
-        for (int z = 0; z < 2; ++z) {
+        for (int z = 0; z < C::kRegions; ++z) {
           tma_load_3d(st + z * C::kRegion, &tmK, &kv_full[s], z * 64, key0, grp);
           tma_load_3d(st + C::kKV + z * C::kRegion, &tmV, &kv_full[s], z * 64, key0, grp);
         }
@@ -866,7 +870,10 @@ __device__ __forceinline__ int decode_cta_of(long long x, const DecodeParams& p)
 // then O in bf16 and LSE.
 constexpr int kMergeRowsPerBlock = 8;
 
+// D / 32 head-dim columns per lane (D = 64 or 128).
+template <int D>
 __global__ void __launch_bounds__(32 * kMergeRowsPerBlock) decode_merge_kernel(const DecodeParams p) {
+  constexpr int kPer = D / 32;
   const long long row = (long long)blockIdx.x * kMergeRowsPerBlock + (threadIdx.x >> 5);
   if (row >= p.rows_total) return;
   const int lane = threadIdx.x & 31;
@@ -876,30 +883,41 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock) decode_merge_kernel(c
   const int i0 = decode_cta_of((long long)G * p.n_chunks, p);
   const int i1 = decode_cta_of((long long)(G + 1) * p.n_chunks - 1, p);
   float m = -INFINITY, wsum = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
 #pragma unroll 4
   for (int i = i0; i <= i1; ++i) {
     const size_t slot_row = (size_t)(G + i) * p.slot_rows + sq;
     const float ls = p.lse_part[slot_row];
-    const float4 o4 = reinterpret_cast<const float4*>(p.o_part + slot_row * 128)[lane];
+    float o[kPer];
+    const float* src = p.o_part + slot_row * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src);
+      o[0] = v.x, o[1] = v.y, o[2] = v.z, o[3] = v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(src);
+      o[0] = v.x, o[1] = v.y;
+    }
     if (ls == -INFINITY) continue;  // no visible key in this segment
     const float m_new = fmaxf(m, ls);
     const float a = __expf(m - m_new);  // 0 while m is still -inf
     const float wgt = __expf(ls - m_new);
     wsum = wsum * a + wgt;
-    acc.x = acc.x * a + wgt * o4.x;
-    acc.y = acc.y * a + wgt * o4.y;
-    acc.z = acc.z * a + wgt * o4.z;
-    acc.w = acc.w * a + wgt * o4.w;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] = acc[e] * a + wgt * o[e];
     m = m_new;
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-  uint2 packed;
-  packed.x = *reinterpret_cast<uint32_t*>(&lo);
-  packed.y = *reinterpret_cast<uint32_t*>(&hi);
-  reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.o) + row * 128)[lane] = packed;
+  uint32_t packed[kPer / 2];
+#pragma unroll
+  for (int e = 0; e < kPer / 2; ++e) packed[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.o) + row * D + lane * kPer;
+  if constexpr (kPer == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = packed[0];
+  }
   if (lane == 0) p.lse[row] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
 }
 
@@ -915,33 +933,41 @@ cudaError_t launch_decode_r(const CUtensorMap& tq, const CUtensorMap& tk, const 
   decode_split_kernel<R><<<(unsigned)p.n_ctas, C::kThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_merge_kernel<<<(unsigned)((p.rows_total + kMergeRowsPerBlock - 1) / kMergeRowsPerBlock),
-                        32 * kMergeRowsPerBlock, 0, s>>>(p);
+  decode_merge_kernel<128><<<(unsigned)((p.rows_total + kMergeRowsPerBlock - 1) / kMergeRowsPerBlock),
+                             32 * kMergeRowsPerBlock, 0, s>>>(p);
   return cudaGetLastError();
 }
 
+template <int D>
 cudaError_t launch_decode_wide(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                const DecodeParams& p, cudaStream_t s) {
-  using C = DecWideCfg;
+  using C = DecWideCfg<D>;
   static std::atomic<uint64_t> configured{0};
-  cudaError_t e = ensure_smem_limit(decode_split_wide_kernel, C::kSmemBytes, configured);
+  cudaError_t e = ensure_smem_limit(decode_split_wide_kernel<D>, C::kSmemBytes, configured);
   if (e != cudaSuccess) return e;
-  decode_split_wide_kernel<<<(unsigned)p.n_ctas, C::kThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
+  decode_split_wide_kernel<D><<<(unsigned)p.n_ctas, C::kThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_merge_kernel<<<(unsigned)((p.rows_total + kMergeRowsPerBlock - 1) / kMergeRowsPerBlock),
-                        32 * kMergeRowsPerBlock, 0, s>>>(p);
+  decode_merge_kernel<D><<<(unsigned)((p.rows_total + kMergeRowsPerBlock - 1) / kMergeRowsPerBlock),
+                           32 * kMergeRowsPerBlock, 0, s>>>(p);
   return cudaGetLastError();
 }
 
-int decode_rows_per_cta(int rows) { return rows <= 16 ? 16 : rows <= 32 ? 32 : DecWideCfg::kBlockRows; }
+// d = 128: groups of up to 32 rows take the kernels with the rows as the MMA's N (the
+// cache read once); larger groups, and every group at d = 64 (whose O^T would need an
+// M = 64 MMA), take 128-row blocks.
+int decode_rows_per_cta(int rows, int d) {
+  if (d != 128) return DecWideCfg<64>::kBlockRows;
+  return rows <= 16 ? 16 : rows <= 32 ? 32 : DecWideCfg<128>::kBlockRows;
+}
 
 cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           cudaStream_t s) {
-  switch (decode_rows_per_cta(p.rows)) {
+  if (p.d == 64) return launch_decode_wide<64>(tq, tk, tv, p, s);
+  switch (decode_rows_per_cta(p.rows, p.d)) {
     case 16: return launch_decode_r<16>(tq, tk, tv, p, s);
     case 32: return launch_decode_r<32>(tq, tk, tv, p, s);
-    default: return launch_decode_wide(tq, tk, tv, p, s);
+    default: return launch_decode_wide<128>(tq, tk, tv, p, s);
   }
 }
 

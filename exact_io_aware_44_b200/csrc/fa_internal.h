@@ -60,7 +60,7 @@ struct DecodeParams {
   float* o_part;      // workspace: per segment slot, normalised partial O [n_slots, slot_rows, d]
   float* lse_part;    // workspace: per segment slot, partial LSE (natural log) [n_slots, slot_rows]
   int* status;
-  int B, Hq, Hkv, Nq, Nk;
+  int B, Hq, Hkv, Nq, Nk, d;
   int causal;
   int rows;                        // query rows of a GQA group: (Hq / Hkv) * Nq
   int n_rb;                        // row blocks per group (units of the chunk sequence)
@@ -86,7 +86,7 @@ cudaError_t launch_fwd_f32(const FwdF32Params& p, cudaStream_t s);
 // Decode: the split kernel, then the merge of the splits.
 // Query rows per decode CTA for a GQA group of `rows` rows: 16 or 32 (one CTA's
 // MMA N covers the group), else 128 (a row block, the MMA M).
-int decode_rows_per_cta(int rows);
+int decode_rows_per_cta(int rows, int d);
 cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           cudaStream_t s);
 // Query rows per tile of the main backward kernel for head dim d (its TMA box height).

@@ -154,10 +154,11 @@ size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, 
  *   num_splits  work split: <= 0 gives one CTA per SM of a 148-SM part; > 0 gives
  *               units*num_splits CTAs (about num_splits key splits per group, or
  *               per row block of 128 rows); never more CTAs than 128-key chunks
- *   d must be 128, else FA_ERR_UNSUPPORTED; causal with Nq > Nk is
- *   FA_ERR_INVALID_ARG. A group of up to 32 query rows is served by one CTA at a
- *   time with the rows as the MMA's N, so its keys are read once; larger groups
- *   take 128-row blocks as the MMA's M, and their keys are read once per block.
+ *   d must be 64 or 128, else FA_ERR_UNSUPPORTED; causal with Nq > Nk is
+ *   FA_ERR_INVALID_ARG. At d = 128 a group of up to 32 query rows is served by
+ *   one CTA at a time with the rows as the MMA's N, so its keys are read once;
+ *   larger groups, and all groups at d = 64, take 128-row blocks as the MMA's M,
+ *   and their keys are read once per block.
  *   Arithmetic: bf16 operands, fp32 accumulation; P is rounded to bf16 before
  *   the P V product; the partials stay fp32.
  */

@@ -86,7 +86,8 @@ def _dec(B=1, Hq=8, Hkv=1, Nq=1, Nk=1000, d=128, causal=1, scale=0.088, splits=0
 
 
 def test_decode_rejects_bad_arguments_on_host():
-    assert _dec(d=64) == -2                        # d = 128 only
+    assert _dec(d=256) == -2                       # d = 64 or 128
+    assert _dec(d=64, ptr=0x1008) == -3            # d = 64: accepted up to the pointer check
     assert _dec(Hq=64, Hkv=1, ptr=0x1008) == -3    # 64 query rows per group: accepted up to the pointer check
     assert _dec(Hq=8, Nq=5, ws=0x1010) == -3       # 40 rows: row blocks, past the size checks
     assert _dec(Hq=16, Nq=3000, Nk=3000, ptr=0x1008) == -3   # 48000 rows: 375 row blocks
@@ -127,7 +128,11 @@ def test_decode_workspace_and_split_rule():
             slots, slot_rows, units = _decode_split(B, Hq, Hkv, Nq, Nk, splits)
             pad = lambda x: (x + 255) // 256 * 256
             assert ws == pad(slots * slot_rows * d * 4) + slots * slot_rows * 4, (B, Hq, Hkv, Nq, Nk, splits, ws)
-    assert fa.decode_workspace_bytes(1, 8, 1, 1, 1000, 64, 0) == 0
+    assert fa.decode_workspace_bytes(1, 8, 1, 1, 1000, 256, 0) == 0
+    # d = 64: the same split rule, d = 64 floats per partial row
+    slots, slot_rows, _ = _decode_split(2, 8, 2, 3, 1000, 0)
+    pad = lambda x: (x + 255) // 256 * 256
+    assert fa.decode_workspace_bytes(2, 8, 2, 3, 1000, 64, 0) == pad(slots * slot_rows * 64 * 4) + slots * slot_rows * 4
 
 
 def test_bwd_rejects_bad_arguments_on_host():

@@ -74,6 +74,26 @@ def test_decode_small(cuda_device, shape, splits, causal):
     check(w, cuda_device, splits)
 
 
+D64_SHAPES = [
+    # B, Hq, Hkv, Nq, Nk: d = 64 takes 128-row blocks for every group size
+    (1, 8, 1, 1, 1),
+    (2, 8, 2, 1, 1000),
+    (1, 32, 4, 4, 2500),    # 32 rows
+    (2, 16, 2, 8, 1300),    # 64 rows
+    (1, 16, 1, 9, 700),     # 144 rows: a full block and a block of 16
+    (3, 8, 2, 1, 7000),     # segments across units
+]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("splits", [0, 3])
+@pytest.mark.parametrize("shape", D64_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_decode_d64(cuda_device, shape, splits, causal):
+    B, Hq, Hkv, Nq, Nk = shape
+    w = synth.DecodeWorkload(f"d64_{'x'.join(map(str, shape))}", B, Hq, Hkv, Nq, Nk, 64, causal, 2600 + Nk + Nq)
+    check(w, cuda_device, splits)
+
+
 def test_decode_square_matches_the_forward(cuda_device):
     """Nq = Nk: the decode mask is fa_fwd's causal mask; both within tolerance of each other."""
     import torch

@@ -1,6 +1,6 @@
 """Seeded random shapes against the oracle: forward and backward over every head
 dim and GQA ratio, decode over every kernel (16 and 32 rows a group, 128-row
-blocks with a partial last block), with ragged lengths that do not line up with
+blocks with a partial last block; d = 64 and 128), with ragged lengths that do not line up with
 the 128-row tiles. The shapes are drawn once from a fixed seed, so every run
 checks the same cases; each case uses the same parity bounds as the targeted
 tests.
@@ -40,7 +40,8 @@ def _decode_cases(n, seed):
         nk = int(rng.integers(nq, 5000))
         causal = bool(rng.integers(0, 2))
         splits = int(rng.choice([0, 0, 1, 5]))
-        cases.append((B, hkv * g, hkv, nq, nk, causal, splits, 8000 + i))
+        d = int(rng.choice([64, 128, 128]))
+        cases.append((B, hkv * g, hkv, nq, nk, causal, splits, d, 8000 + i))
     return cases
 
 
@@ -63,13 +64,13 @@ def test_random_attention_fwd_bwd(cuda_device, case):
         assert rel_fro(a.float().cpu().numpy(), ref) <= BWD_REL_FRO, (name, case)
 
 
-@pytest.mark.parametrize("case", _decode_cases(24, 20261204), ids=lambda c: "x".join(map(str, c[:7])))
+@pytest.mark.parametrize("case", _decode_cases(24, 20261204), ids=lambda c: "x".join(map(str, c[:8])))
 def test_random_decode(cuda_device, case):
     import torch
 
     import exact_io_aware_44_b200 as fa
-    B, Hq, Hkv, Nq, Nk, causal, splits, seed = case
-    w = synth.DecodeWorkload("fz", B, Hq, Hkv, Nq, Nk, 128, causal, seed)
+    B, Hq, Hkv, Nq, Nk, causal, splits, d, seed = case
+    w = synth.DecodeWorkload("fz", B, Hq, Hkv, Nq, Nk, d, causal, seed)
     q, k, v = synth.decode_inputs(w)
     o, lse = fa.decode(*(to_dev(x, torch.bfloat16, cuda_device) for x in (q, k, v)), causal=causal,
                        num_splits=splits)
