@@ -54,9 +54,9 @@ NCU_TRAFFIC = {
     ("fwd", "c3"): {"bytes_per_launch": 403261696 + 118636032, "csrc_sha": "3b3769599fbeb05b"},
     ("fwd", "c4"): {"bytes_per_launch": 811248896 + 262354432, "csrc_sha": "3b3769599fbeb05b"},
     # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md, profiles/decode_wide_B16Hq64Hkv8Nq8_Nk32768_d128.md
-    ("decode_split", "dec"): {"bytes_per_launch": 2148271104 + 3724800, "csrc_sha": "0bd30d5eb481de28"},
-    ("decode_split", "dec4"): {"bytes_per_launch": 1074862848 + 4931584, "csrc_sha": "0bd30d5eb481de28"},
-    ("decode_split", "dec8"): {"bytes_per_launch": 2153814528 + 8017408, "csrc_sha": "0bd30d5eb481de28"},
+    ("decode_split", "dec"): {"bytes_per_launch": 2148459264 + 3497728, "csrc_sha": "91306dfb6f4e6182"},
+    ("decode_split", "dec4"): {"bytes_per_launch": 1074816512 + 4360448, "csrc_sha": "91306dfb6f4e6182"},
+    ("decode_split", "dec8"): {"bytes_per_launch": 2153745920 + 7677696, "csrc_sha": "91306dfb6f4e6182"},
 }
 
 
