@@ -62,8 +62,12 @@ __device__ __forceinline__ void red_add(float* p, float a) {
 }
 
 // ---------------------------------------------------------------------------
-// D = rowsum(dO o O); dQ accumulator = 0. One thread per 8 columns of a row.
+// D = rowsum(dO o O); dQ accumulator = 0. One thread per 8 columns of a row, and
+// kPrepItems such (row, 8 columns) items per thread per round, whose loads are all
+// issued before any is used (more bytes in flight per thread).
 // ---------------------------------------------------------------------------
+constexpr int kPrepItems = 4;
+
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
                                                              const __nv_bfloat16* __restrict__ dout,
@@ -71,48 +75,79 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
                                                              long long rows) {
   constexpr int kPer = D / 8;  // threads per row (32, 16 or 8)
   const long long total = rows * kPer;
-  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t - threadIdx.x < total;
-       t += (long long)gridDim.x * blockDim.x) {
-    const bool in = t < total;
-    const long long row = t / kPer;
-    const int part = (int)(t % kPer);
-    float acc = 0.f;
-    if (in) {
-      const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
-      const uint4 b = *reinterpret_cast<const uint4*>(dout + row * D + part * 8);
-      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  // rounds are taken by whole warps (t - threadIdx.x is the same across a block), so the
+  // shuffles below always see converged warps
+  for (long long t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; t0 - threadIdx.x < total;
+       t0 += kPrepItems * stride) {
+    uint4 a[kPrepItems], b[kPrepItems];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 x = __bfloat1622float2(a2[i]);
-        const float2 y = __bfloat1622float2(b2[i]);
-        acc = fmaf(x.x, y.x, acc);
-        acc = fmaf(x.y, y.y, acc);
+    for (int j = 0; j < kPrepItems; ++j) {
+      const long long t = t0 + j * stride;
+      if (t < total) {
+        const long long row = t / kPer;
+        const int part = (int)(t % kPer);
+        a[j] = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
+        b[j] = *reinterpret_cast<const uint4*>(dout + row * D + part * 8);
       }
-      float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
-      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int off = kPer / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (in && part == 0) delta[row] = acc;
+    for (int j = 0; j < kPrepItems; ++j) {
+      const long long t = t0 + j * stride;
+      const bool in = t < total;
+      const long long row = t / kPer;
+      const int part = (int)(t % kPer);
+      float acc = 0.f;
+      if (in) {
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a[j]);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b[j]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 x = __bfloat1622float2(a2[i]);
+          const float2 y = __bfloat1622float2(b2[i]);
+          acc = fmaf(x.x, y.x, acc);
+          acc = fmaf(x.y, y.y, acc);
+        }
+        float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int off = kPer / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (in && part == 0) delta[row] = acc;
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
-// dQ = bf16(scale * accumulator), 8 elements per thread.
+// dQ = bf16(scale * accumulator), 8 elements per item, kPrepItems items per thread
+// per round with all their loads in flight together.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) bwd_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
                                                           long long n8, float scale) {
-  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n8; t += (long long)gridDim.x * blockDim.x) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * t];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * t + 1];
-    uint4 u;
-    u.x = pack_bf16x2(a.x * scale, a.y * scale);
-    u.y = pack_bf16x2(a.z * scale, a.w * scale);
-    u.z = pack_bf16x2(b.x * scale, b.y * scale);
-    u.w = pack_bf16x2(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dq)[t] = u;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; t0 < n8; t0 += kPrepItems * stride) {
+    float4 a[kPrepItems], b[kPrepItems];
+#pragma unroll
+    for (int j = 0; j < kPrepItems; ++j) {
+      const long long t = t0 + j * stride;
+      if (t < n8) {
+        a[j] = reinterpret_cast<const float4*>(acc)[2 * t];
+        b[j] = reinterpret_cast<const float4*>(acc)[2 * t + 1];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kPrepItems; ++j) {
+      const long long t = t0 + j * stride;
+      if (t < n8) {
+        uint4 u;
+        u.x = pack_bf16x2(a[j].x * scale, a[j].y * scale);
+        u.y = pack_bf16x2(a[j].z * scale, a[j].w * scale);
+        u.z = pack_bf16x2(b[j].x * scale, b[j].y * scale);
+        u.w = pack_bf16x2(b[j].z * scale, b[j].w * scale);
+        reinterpret_cast<uint4*>(dq)[t] = u;
+      }
+    }
   }
 }
 
@@ -1060,7 +1095,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 template <int D>
 cudaError_t launch_preprocess_d(const BwdParams& p, cudaStream_t s) {
   const long long rows = (long long)p.B * p.Hq * p.N;
-  const int blocks = (int)std::min<long long>((rows * (D / 8) + 255) / 256, 8LL * sm_count());
+  const int blocks = (int)std::min<long long>((rows * (D / 8) + 256 * kPrepItems - 1) / (256 * kPrepItems),
+                                              8LL * sm_count());
   bwd_preprocess_kernel<D><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(p.o),
                                                    static_cast<const __nv_bfloat16*>(p.dout), p.delta, p.dq_acc, rows);
   return cudaGetLastError();
@@ -1549,7 +1585,7 @@ cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const 
 
 cudaError_t launch_bwd_convert(const BwdParams& p, cudaStream_t s) {
   const long long n8 = (long long)p.B * p.Hq * p.N * p.d / 8;
-  const int blocks = (int)std::min<long long>((n8 + 255) / 256, 8LL * sm_count());
+  const int blocks = (int)std::min<long long>((n8 + 256 * kPrepItems - 1) / (256 * kPrepItems), 8LL * sm_count());
   bwd_convert_kernel<<<blocks, 256, 0, s>>>(p.dq_acc, static_cast<__nv_bfloat16*>(p.dq), n8, p.scale);
   return cudaGetLastError();
 }
