@@ -49,7 +49,7 @@ NCU_TRAFFIC = {
     # profiles/bwd_main_d128_B2H32N8192_causal.md
     ("bwd_main", "c3"): {"bytes_per_launch": 810053376 + 491489280, "csrc_sha": "eca1cf4d70f597f7"},
     # profiles/bwd_main_d64_B4H16N2048_causal.md
-    ("bwd_main", "c2"): {"bytes_per_launch": 101785600 + 24538112, "csrc_sha": "e795a43c1c31fa93"},
+    ("bwd_main", "c2"): {"bytes_per_launch": 101785600 + 24538112, "csrc_sha": "0db9771b218176f6"},
     # profiles/fwd_bf16_d128_B2H32N8192_causal.md
     ("fwd", "c3"): {"bytes_per_launch": 403261696 + 118636032, "csrc_sha": "3b3769599fbeb05b"},
     ("fwd", "c4"): {"bytes_per_launch": 811248896 + 262354432, "csrc_sha": "3b3769599fbeb05b"},
@@ -66,7 +66,7 @@ NCU_TRAFFIC = {
 KERNEL_SOURCES = {
     "bwd_main": ("fa_bwd_sm100.cu", [("__device__ __forceinline__ void red_add(", "// ----"),
                                      ("struct Bwd128Cfg {", "struct Bwd64Cfg {")]),
-    "bwd_main_d64": ("fa_bwd_sm100.cu", [("struct Bwd64Cfg {", "cudaError_t launch_main_d128(")]),
+    "bwd_main_d64": ("fa_bwd_sm100.cu", [("struct Bwd64Cfg {", "template <int D>\ncudaError_t launch_preprocess_d(")]),
     "fwd": ("fa_fwd_sm100.cu", [("", None)]),
     "decode_split": ("fa_decode_sm100.cu", [("template <int R>\nstruct DecCfg {", "template <int R>\ncudaError_t launch_decode_r(")]),
 }
