@@ -82,6 +82,10 @@ struct FwdCfg {
   static constexpr int kElem = FP8 ? 1 : 2;                      // bytes per element
   // Query tiles per CTA: two, except d = 256, whose O tile alone takes 256 TMEM columns.
   static constexpr int kTiles = D == 256 ? 1 : 2;
+  // One tile per CTA leaves nothing to overlap the chain P(j) -> P V(j) -> S(j+1), so there
+  // the softmax hands over the first 64 keys of P(j) while it exponentiates the rest and the
+  // P V product runs in two halves (with two tiles the mid-tile hand-off only slowed it).
+  static constexpr bool kSplitPV = !FP8 && kTiles == 1;
   // K/V ring: K_0, V_0, K_1, V_1, ... (d = 256: two 64 KB stages next to the 64 KB Q tile)
   static constexpr int kStages = (FP8 || D == 64) ? 10 : (D == 256 ? 2 : 5);
   static constexpr int kTileBytes = kTileM * D * kElem;          // one Q, K or V tile
@@ -94,8 +98,8 @@ struct FwdCfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kOffQ + kTiles * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  // q_full, q_empty, full[S], empty[S], s_ready[2], p_ready[2], o_done[2], mma_final
-  static constexpr int kNumBars = 2 + 2 * kStages + 7;
+  // q_full, q_empty, full[S], empty[S], s_ready[2], p_ready[2], o_done[2], mma_final, p_half[2]
+  static constexpr int kNumBars = 2 + 2 * kStages + 9;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
 };
@@ -189,6 +193,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* p_ready = s_ready + 2;
   uint64_t* o_done = p_ready + 2;
   uint64_t* mma_final = o_done + 2;
+  uint64_t* p_half = mma_final + 1;  // kSplitPV: keys [0, 64) of P_t stored
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -207,6 +212,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&s_ready[t], 1);
       mbar_init(&p_ready[t], kTileM);
       mbar_init(&o_done[t], 1);
+      mbar_init(&p_half[t], kTileM);
     }
     mbar_init(mma_final, 1);
     *abort_flag = 0;
@@ -309,10 +315,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (leader) mma_commit(&s_ready[t]);
     };
-    auto issue_pv = [&](int t, int slot, int j) {
+    auto issue_pv = [&](int t, int slot, int j, int k_lo, int k_hi) {  // K steps [k_lo, k_hi)
       const uint64_t b0 = desc_advance(d_v, slot * C::kTileBytes);
 #pragma unroll
-      for (int k = 0; k < C::kPvSteps; ++k) {
+      for (int k = k_lo; k < k_hi; ++k) {
         if (leader) {
           const uint64_t bk = desc_advance(b0, k * C::kKStep * 128);
           if constexpr (FP8)
@@ -351,10 +357,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t) {  // unrolled: t, the TMEM columns and barriers are constants
           if (j >= U.n_iter[t]) continue;
+          constexpr int kPvFirst = C::kSplitPV ? C::kPvSteps / 2 : 0;
+          if constexpr (C::kSplitPV) {  // keys [0, 64) of P_t as soon as they are stored
+            if (!(ok = warp_wait_spin(&p_half[t], (p_base[t] + j) & 1, w))) break;
+            tc_fence_after();
+            issue_pv(t, vslot, j, 0, kPvFirst);
+          }
           if (!(ok = warp_wait_spin(&p_ready[t], (p_base[t] + j) & 1, w))) break;
           if (leader && prog) prog[blockIdx.x] = (unsigned)(++pv_count);
           tc_fence_after();
-          issue_pv(t, vslot, j);
+          issue_pv(t, vslot, j, kPvFirst, C::kPvSteps);
           if (j + 1 < U.n_iter[t]) {
             if (kslot < 0 && !(ok = take(kslot))) break;
             issue_s(t, kslot);
@@ -451,6 +463,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           rescale = true;
         }
         const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+        // PV(j-1) has completed (the commit of S(j) covers it): O may be rescaled, which
+        // must happen before any of P(j) is handed to the P V product.
+        auto rescale_o = [&]() {
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t r[32];
+              tmem_ld32(tO + cc * 32, r);
+              tmem_ld_wait(r);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+              tmem_st32(tO + cc * 32, r);
+            }
+          }
+        };
         // P = 2^(S c - m c), packed at once (bf16 pairs, or E4M3 quads: one TMEM column
         // each); l sums the fp32 values. P <= 2^8 fits E4M3; E4M3 flushes P < 2^-10 to zero.
         uint32_t pk[kTileN / (FP8 ? 4 : 2)];
@@ -483,6 +510,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           } else {
             pk[i / 2] = pack_bf16x2(e0, e1);
             pk[i / 2 + 1] = pack_bf16x2(e2, e3);
+            if (C::kSplitPV && i + 4 == kTileN / 2) {  // keys [0, 64) done: hand them over
+              rescale_o();
+              tmem_st32(tS, *reinterpret_cast<uint32_t (*)[32]>(&pk[0]));
+              tmem_st_wait();
+              tc_fence_before();
+              mbar_arrive(&p_half[t]);
+            }
           }
         }
         float ra, rb, rc, rd;
@@ -490,26 +524,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         f2_unpack(rs2[1], rc, rd);
         l += (ra + rb) + (rc + rd);
 
-        // PV(j-1) has completed (the commit of S(j) covers it): O may be rescaled.
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t r[32];
-            tmem_ld32(tO + cc * 32, r);
-            tmem_ld_wait(r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(tO + cc * 32, r);
-          }
-        }
+        if constexpr (!C::kSplitPV) rescale_o();
         // P into the first columns of S_t (its scores are in registers now).
         if constexpr (FP8) {
           tmem_st32(tS, pk);
         } else {
-          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[0]);
-          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[32]);
-          tmem_st32(tS, lo);
-          tmem_st32(tS + 32, hi);
+          if constexpr (!C::kSplitPV) tmem_st32(tS, *reinterpret_cast<uint32_t (*)[32]>(&pk[0]));
+          tmem_st32(tS + 32, *reinterpret_cast<uint32_t (*)[32]>(&pk[32]));
         }
         tmem_st_wait();
         tc_fence_before();
