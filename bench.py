@@ -50,9 +50,10 @@ NCU_TRAFFIC = {
     ("bwd_main", "c3"): {"bytes_per_launch": 810053376 + 491489280, "csrc_sha": "eca1cf4d70f597f7"},
     # profiles/bwd_main_d64_B4H16N2048_causal.md
     ("bwd_main", "c2"): {"bytes_per_launch": 101785600 + 24538112, "csrc_sha": "0db9771b218176f6"},
-    # profiles/fwd_bf16_d128_B2H32N8192_causal.md
-    ("fwd", "c3"): {"bytes_per_launch": 403261696 + 118636032, "csrc_sha": "3b3769599fbeb05b"},
-    ("fwd", "c4"): {"bytes_per_launch": 811248896 + 262354432, "csrc_sha": "3b3769599fbeb05b"},
+    # profiles/fwd_bf16_d128_B2H32N8192_causal.md, profiles/fwd_bf16_d256_B2H16N8192_causal.md
+    ("fwd", "c3"): {"bytes_per_launch": 404125696 + 117713664, "csrc_sha": "6c7ab7a7c997f0df"},
+    ("fwd", "c4"): {"bytes_per_launch": 810168320 + 260882688, "csrc_sha": "6c7ab7a7c997f0df"},
+    ("fwd", "c6"): {"bytes_per_launch": 403628032 + 119477504, "csrc_sha": "6c7ab7a7c997f0df"},
     # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md, profiles/decode_wide_B16Hq64Hkv8Nq8_Nk32768_d128.md
     ("decode_split", "dec"): {"bytes_per_launch": 2148459264 + 3497728, "csrc_sha": "91306dfb6f4e6182"},
     ("decode_split", "dec4"): {"bytes_per_launch": 1074816512 + 4360448, "csrc_sha": "91306dfb6f4e6182"},
