@@ -8,7 +8,7 @@
 // matrix only ever exists as one 128 x 128 tile in Tensor Memory.
 //
 // The kernel is persistent: one CTA per SM, 384 threads, looping over work units
-// of two 128-row query tiles of one (batch, head) (one tile at d = 256). Units are
+// of two 128-row query tiles of one (batch, head). Units are
 // dealt to the CTAs in rounds, in snake order over a heavy-first list; Tensor
 // Memory, the barriers and the K/V ring stay set up from one unit to the next,
 // and the next unit's Q and K/V loads overlap the current unit's last tiles.
@@ -45,6 +45,9 @@
 // PV_t(j), so when a softmax warpgroup sees S_t(j+1), O_t is complete and may be
 // rescaled. While one softmax warpgroup exponentiates, the tensor core runs the
 // other tile's P V and scores.
+//
+// d = 256 (fwd256_kernel, further down): the O tile alone takes 256 columns, so a
+// CTA holds one query tile, and the spare 128 columns double-buffer its scores.
 #include <math.h>
 
 #include <algorithm>
@@ -80,14 +83,10 @@ constexpr int kPolyPairs64 = FA_FWD64_POLY_PAIRS;  // the same, for d = 64 (bf16
 template <int D, bool FP8>
 struct FwdCfg {
   static constexpr int kElem = FP8 ? 1 : 2;                      // bytes per element
-  // Query tiles per CTA: two, except d = 256, whose O tile alone takes 256 TMEM columns.
-  static constexpr int kTiles = D == 256 ? 1 : 2;
-  // One tile per CTA leaves nothing to overlap the chain P(j) -> P V(j) -> S(j+1), so there
-  // the softmax hands over the first 64 keys of P(j) while it exponentiates the rest and the
-  // P V product runs in two halves (with two tiles the mid-tile hand-off only slowed it).
-  static constexpr bool kSplitPV = !FP8 && kTiles == 1;
-  // K/V ring: K_0, V_0, K_1, V_1, ... (d = 256: two 64 KB stages next to the 64 KB Q tile)
-  static constexpr int kStages = (FP8 || D == 64) ? 10 : (D == 256 ? 2 : 5);
+  static_assert(D == 64 || D == 128, "d = 256 has a kernel of its own (fwd256_kernel)");
+  static constexpr int kTiles = 2;  // query tiles per CTA
+  // K/V ring: K_0, V_0, K_1, V_1, ...
+  static constexpr int kStages = (FP8 || D == 64) ? 10 : 5;
   static constexpr int kTileBytes = kTileM * D * kElem;          // one Q, K or V tile
   static constexpr int kRegion = kTileM * 128;                   // one 128-byte-wide column block
   static constexpr int kRegions = D * kElem / 128;               // column blocks per tile
@@ -98,8 +97,8 @@ struct FwdCfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kOffQ + kTiles * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  // q_full, q_empty, full[S], empty[S], s_ready[2], p_ready[2], o_done[2], mma_final, p_half[2]
-  static constexpr int kNumBars = 2 + 2 * kStages + 9;
+  // q_full, q_empty, full[S], empty[S], s_ready[2], p_ready[2], o_done[2], mma_final
+  static constexpr int kNumBars = 2 + 2 * kStages + 7;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
 };
@@ -193,7 +192,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* p_ready = s_ready + 2;
   uint64_t* o_done = p_ready + 2;
   uint64_t* mma_final = o_done + 2;
-  uint64_t* p_half = mma_final + 1;  // kSplitPV: keys [0, 64) of P_t stored
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -212,7 +210,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&s_ready[t], 1);
       mbar_init(&p_ready[t], kTileM);
       mbar_init(&o_done[t], 1);
-      mbar_init(&p_half[t], kTileM);
     }
     mbar_init(mma_final, 1);
     *abort_flag = 0;
@@ -315,10 +312,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (leader) mma_commit(&s_ready[t]);
     };
-    auto issue_pv = [&](int t, int slot, int j, int k_lo, int k_hi) {  // K steps [k_lo, k_hi)
+    auto issue_pv = [&](int t, int slot, int j) {
       const uint64_t b0 = desc_advance(d_v, slot * C::kTileBytes);
 #pragma unroll
-      for (int k = k_lo; k < k_hi; ++k) {
+      for (int k = 0; k < C::kPvSteps; ++k) {
         if (leader) {
           const uint64_t bk = desc_advance(b0, k * C::kKStep * 128);
           if constexpr (FP8)
@@ -357,16 +354,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t) {  // unrolled: t, the TMEM columns and barriers are constants
           if (j >= U.n_iter[t]) continue;
-          constexpr int kPvFirst = C::kSplitPV ? C::kPvSteps / 2 : 0;
-          if constexpr (C::kSplitPV) {  // keys [0, 64) of P_t as soon as they are stored
-            if (!(ok = warp_wait_spin(&p_half[t], (p_base[t] + j) & 1, w))) break;
-            tc_fence_after();
-            issue_pv(t, vslot, j, 0, kPvFirst);
-          }
           if (!(ok = warp_wait_spin(&p_ready[t], (p_base[t] + j) & 1, w))) break;
           if (leader && prog) prog[blockIdx.x] = (unsigned)(++pv_count);
           tc_fence_after();
-          issue_pv(t, vslot, j, kPvFirst, C::kPvSteps);
+          issue_pv(t, vslot, j);
           if (j + 1 < U.n_iter[t]) {
             if (kslot < 0 && !(ok = take(kslot))) break;
             issue_s(t, kslot);
@@ -463,21 +454,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           rescale = true;
         }
         const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-        // PV(j-1) has completed (the commit of S(j) covers it): O may be rescaled, which
-        // must happen before any of P(j) is handed to the P V product.
-        auto rescale_o = [&]() {
-          if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-              uint32_t r[32];
-              tmem_ld32(tO + cc * 32, r);
-              tmem_ld_wait(r);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-              tmem_st32(tO + cc * 32, r);
-            }
-          }
-        };
         // P = 2^(S c - m c), packed at once (bf16 pairs, or E4M3 quads: one TMEM column
         // each); l sums the fp32 values. P <= 2^8 fits E4M3; E4M3 flushes P < 2^-10 to zero.
         uint32_t pk[kTileN / (FP8 ? 4 : 2)];
@@ -510,13 +486,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           } else {
             pk[i / 2] = pack_bf16x2(e0, e1);
             pk[i / 2 + 1] = pack_bf16x2(e2, e3);
-            if (C::kSplitPV && i + 4 == kTileN / 2) {  // keys [0, 64) done: hand them over
-              rescale_o();
-              tmem_st32(tS, *reinterpret_cast<uint32_t (*)[32]>(&pk[0]));
-              tmem_st_wait();
-              tc_fence_before();
-              mbar_arrive(&p_half[t]);
-            }
           }
         }
         float ra, rb, rc, rd;
@@ -524,13 +493,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         f2_unpack(rs2[1], rc, rd);
         l += (ra + rb) + (rc + rd);
 
-        if constexpr (!C::kSplitPV) rescale_o();
+        // PV(j-1) has completed (the commit of S(j) covers it): O may be rescaled.
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld32(tO + cc * 32, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(tO + cc * 32, r);
+          }
+        }
         // P into the first columns of S_t (its scores are in registers now).
         if constexpr (FP8) {
           tmem_st32(tS, pk);
         } else {
-          if constexpr (!C::kSplitPV) tmem_st32(tS, *reinterpret_cast<uint32_t (*)[32]>(&pk[0]));
-          tmem_st32(tS + 32, *reinterpret_cast<uint32_t (*)[32]>(&pk[32]));
+          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[0]);
+          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[32]);
+          tmem_st32(tS, lo);
+          tmem_st32(tS + 32, hi);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -575,6 +557,343 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
+// ----------------------------------------------------------------------------
+// fwd256_kernel (bf16, d = 256): one 128-row query tile per CTA, one CTA per unit.
+// The O tile takes 256 TMEM columns, which leaves room for two score buffers, so the
+// scores of key tile j+1 are computed while the softmax works on tile j, and the
+// chain P(j) -> P V(j) -> S(j+1) -> softmax(j+1) of the one-buffer design leaves the
+// critical path: the softmax runs back to back while the tensor core does P V(j-1)
+// and S(j+1) beside it.
+//   TMEM: S buffers [0,128) and [128,256) (key tile parity), O [256,512).
+//   warp 0      TMA producer: Q (64 KB), then K and V in 32 KB halves (128 of the
+//               256 columns) through a ring of 5 stages, in the order the MMAs use
+//               them: K_0, K_1, V_0, K_2, V_1, K_3, ...
+//   warp 1      MMA issuer: S(0), S(1); then per key tile j, once P(j) is stored,
+//               O += P(j) V_j (two N = 128 halves per K step) and S(j+2) into the
+//               buffer P(j) came from (issued after P V(j), and one thread's MMAs run
+//               in issue order).
+//   warps 4-7   softmax (thread = query row = TMEM lane), as in fwd_kernel; before it
+//               stores P(j) it waits for P V(j-1) to finish (which it normally already
+//               has), so that O may be rescaled.
+// P (bf16 pairs, 64 columns) overwrites the first half of its S buffer.
+struct Fwd256Cfg {
+  static constexpr int D = 256;
+  static constexpr int kRegion = kTileM * 128;     // 16 KB: 128 rows x 64 columns (128-byte swizzle)
+  static constexpr int kHalf = 2 * kRegion;        // 32 KB: 128 columns of a K or V tile
+  static constexpr int kStages = 5;
+  static constexpr int kOffQ = 0;                  // Q: 4 regions
+  static constexpr int kOffKV = 4 * kRegion;
+  static constexpr int kOffBar = kOffKV + kStages * kHalf;
+  // q_full, full[S], empty[S], s_ready[2], p_ready, o_ready, mma_final
+  static constexpr int kNumBars = 1 + 2 * kStages + 5;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+};
+
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fwd256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = Fwd256Cfg;
+  constexpr int S = C::kStages;
+  constexpr int D = C::D;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* ring_full = bars + 1;
+  uint64_t* ring_empty = ring_full + S;
+  uint64_t* s_ready = ring_empty + S;
+  uint64_t* p_ready = s_ready + 2;
+  uint64_t* o_ready = p_ready + 1;
+  uint64_t* mma_final = o_ready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const FwdUnit U = fwd_unit<1>(p, (int)blockIdx.x);
+  const int n = U.n_iter[0];  // key tiles of this query tile (>= 1: the tile starts below N)
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&ring_full[s], 1);
+      mbar_init(&ring_empty[s], 1);
+    }
+    mbar_init(&s_ready[0], 1);
+    mbar_init(&s_ready[1], 1);
+    mbar_init(p_ready, kTileM);
+    mbar_init(o_ready, 1);
+    mbar_init(mma_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx w{abort_flag, p.status, p.wait_budget_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    regs_dec<kRegsControl, kRegsLaunch>();
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(q_full, 4 * C::kRegion);
+#pragma unroll
+      for (int z = 0; z < 4; ++z)
+        tma_load_3d(smem + C::kOffQ + z * C::kRegion, &tmQ, q_full, z * 64, U.q0, U.b * p.Hq + U.h);
+      int it = 0;
+      // one K or V tile: its two 32 KB halves, each in a stage of its own
+      auto push = [&](const CUtensorMap* map, int kv_tile) -> bool {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int s = it % S;
+          if (!mbar_wait_spin(&ring_empty[s], ((it / S) & 1) ^ 1, w)) return false;
+          mbar_arrive_expect_tx(&ring_full[s], C::kHalf);
+#pragma unroll
+          for (int z = 0; z < 2; ++z)
+            tma_load_3d(smem + C::kOffKV + s * C::kHalf + z * C::kRegion, map, &ring_full[s], (half * 2 + z) * 64,
+                        kv_tile * kTileN, U.kv_head);
+          ++it;
+        }
+        return true;
+      };
+      bool ok = push(&tmK, 0);
+      if (ok && n > 1) ok = push(&tmK, 1);
+      for (int j = 0; j < n && ok; ++j) {
+        ok = push(&tmV, j);
+        if (ok && j + 2 < n) ok = push(&tmK, j + 2);
+      }
+      if (!ok) {
+        // Error path: let the loads already issued land before the CTA exits.
+        WaitCtx drain{abort_flag, p.status, 20000000ull};
+        volatile int zero = 0;
+        drain.abort_flag = &zero;
+        for (int kk = max(0, it - S); kk < it; ++kk) mbar_wait(&ring_full[kk % S], (kk / S) & 1, drain);
+        mbar_wait(q_full, 0, drain);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    regs_dec<kRegsControl, kRegsLaunch>();
+    const bool leader = lane == 0;
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, 128, false, true);  // one 128-column half of O
+    const uint64_t d_q = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+    const uint64_t d_k = sdesc_sw128(smem_u32(smem + C::kOffKV), 16, 1024);          // K-major view
+    const uint64_t d_v = sdesc_sw128(smem_u32(smem + C::kOffKV), C::kRegion, 1024);  // MN-major view
+    int cnt = 0;
+    auto take = [&](int& slot) -> bool {  // next stage of the ring
+      slot = cnt % S;
+      const bool res = warp_wait_spin(&ring_full[slot], (cnt / S) & 1, w);
+      ++cnt;
+      tc_fence_after();
+      return res;
+    };
+    // S(j) = Q K_j^T into buffer buf: 16 K steps, the first 8 from K's first half
+    auto issue_s = [&](int buf) -> bool {
+      int sa, sb;
+      if (!take(sa) || !take(sb)) return false;
+      const uint64_t ka = desc_advance(d_k, sa * C::kHalf), kb = desc_advance(d_k, sb * C::kHalf);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const uint32_t qoff = (k >> 2) * C::kRegion + (k & 3) * 32;
+        const uint32_t koff = ((k >> 2) & 1) * C::kRegion + (k & 3) * 32;
+        if (leader)
+          mma_bf16_ss(tmem + buf * 128, desc_advance(d_q, qoff), desc_advance(k < 8 ? ka : kb, koff), kIdescS,
+                      k > 0 ? 1u : 0u);
+      }
+      if (leader) {
+        mma_commit(&s_ready[buf]);
+        mma_commit(&ring_empty[sa]);
+        mma_commit(&ring_empty[sb]);
+      }
+      return true;
+    };
+    // O += P(j) V_j: P from buffer buf, V's halves give O's column halves
+    auto issue_pv = [&](int buf, int j) -> bool {
+      int sa, sb;
+      if (!take(sa) || !take(sb)) return false;
+      const uint64_t va = desc_advance(d_v, sa * C::kHalf), vb = desc_advance(d_v, sb * C::kHalf);
+#pragma unroll
+      for (int k = 0; k < kTileN / 16; ++k) {
+        if (leader) {
+          const uint32_t acc = (j > 0 || k > 0) ? 1u : 0u;
+          mma_bf16_ts(tmem + 256, tmem + buf * 128 + k * 8, desc_advance(va, k * 16 * 128), kIdescPV, acc);
+          mma_bf16_ts(tmem + 384, tmem + buf * 128 + k * 8, desc_advance(vb, k * 16 * 128), kIdescPV, acc);
+        }
+      }
+      if (leader) {
+        mma_commit(o_ready);
+        mma_commit(&ring_empty[sa]);
+        mma_commit(&ring_empty[sb]);
+      }
+      return true;
+    };
+    unsigned* const prog = (int)blockIdx.x < p.progress_n ? p.progress : nullptr;
+    if (leader && prog) prog[blockIdx.x] = 0u;
+    bool ok = warp_wait_spin(q_full, 0, w);
+    tc_fence_after();
+    if (ok) ok = issue_s(0);
+    if (ok && n > 1) ok = issue_s(1);
+    for (int j = 0; j < n && ok; ++j) {
+      if (!(ok = warp_wait_spin(p_ready, j & 1, w))) break;
+      tc_fence_after();
+      if (leader && prog) prog[blockIdx.x] = (unsigned)(j + 1);
+      if (!(ok = issue_pv(j & 1, j))) break;
+      if (j + 2 < n) ok = issue_s(j & 1);
+    }
+    // Every MMA issued above must finish before TMEM is released.
+    if (leader) mma_commit(mma_final);
+    __syncwarp();
+    WaitCtx drain{abort_flag, p.status, 20000000ull};
+    volatile int zero = 0;
+    drain.abort_flag = &zero;
+    mbar_wait(mma_final, 0, drain);
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ softmax
+    regs_inc<kRegsSoftmax, kRegsLaunch>();
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tO = tmem + lane_off + 256;
+    const float c = p.scale_log2;
+    const int qrow = U.q0 + row;
+    float m_ref = -INFINITY;  // reference max (raw score units)
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int buf = j & 1;
+      const uint32_t tS = tmem + lane_off + buf * 128;
+      if (!(ok = consumer_wait(&s_ready[buf], (j >> 1) & 1, w))) break;
+      tc_fence_after();
+      float s[kTileN];
+#pragma unroll
+      for (int cc = 0; cc < kTileN / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tS + cc * 32, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
+      }
+      const int k0 = j * kTileN;
+      if (p.causal && j == n - 1) {
+        const int lim = qrow - k0;  // keys with column > lim are in the future
+#pragma unroll
+        for (int i = 0; i < kTileN; ++i)
+          if (i > lim) s[i] = -INFINITY;
+      } else if (!p.causal && j == n - 1 && p.N - k0 < kTileN) {
+        const int lim = p.N - k0;
+#pragma unroll
+        for (int i = 0; i < kTileN; ++i)
+          if (i >= lim) s[i] = -INFINITY;
+      }
+      float mq[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+      for (int i = 4; i < kTileN; i += 8) {
+        mq[0] = fmax3(mq[0], s[i], s[i + 1]);
+        mq[1] = fmax3(mq[1], s[i + 2], s[i + 3]);
+        mq[2] = fmax3(mq[2], s[i + 4], s[i + 5]);
+        if (i + 6 < kTileN) mq[3] = fmax3(mq[3], s[i + 6], s[i + 7]);
+      }
+      const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
+      const float m_new = fmaxf(m_ref, mx);
+      float alpha = 1.f;
+      bool rescale = false;
+      if (j == 0) {
+        m_ref = m_new;
+      } else if ((m_new - m_ref) * c > (float)kRescaleThresholdLog2) {
+        alpha = ex2((m_ref - m_new) * c);
+        m_ref = m_new;
+        l *= alpha;
+        rescale = true;
+      }
+      const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+      uint32_t pk[kTileN / 2];
+      uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+      const uint64_t c2 = f2_pack(c, c), nmc2 = f2_pack(-mc, -mc);
+#pragma unroll
+      for (int i = 0; i < kTileN; i += 4) {
+        float x0, x1, x2, x3;
+        f2_unpack(f2_fma(f2_pack(s[i], s[i + 1]), c2, nmc2), x0, x1);
+        f2_unpack(f2_fma(f2_pack(s[i + 2], s[i + 3]), c2, nmc2), x2, x3);
+        const float e0 = ex2(x0), e1 = ex2(x1), e2 = ex2(x2), e3 = ex2(x3);
+        rs2[0] = f2_add(rs2[0], f2_pack(e0, e1));
+        rs2[1] = f2_add(rs2[1], f2_pack(e2, e3));
+        pk[i / 2] = pack_bf16x2(e0, e1);
+        pk[i / 2 + 1] = pack_bf16x2(e2, e3);
+      }
+      float ra, rb, rc, rd;
+      f2_unpack(rs2[0], ra, rb);
+      f2_unpack(rs2[1], rc, rd);
+      l += (ra + rb) + (rc + rd);
+      // P V(j-1) must be done before O is rescaled; it was issued a whole softmax ago.
+      if (j > 0) {
+        if (!(ok = consumer_wait(o_ready, (j - 1) & 1, w))) break;
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(tO + cc * 32, r);
+          tmem_ld_wait(r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(tO + cc * 32, r);
+        }
+      }
+      tmem_st32(tS, *reinterpret_cast<uint32_t (*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t (*)[32]>(&pk[32]));
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+    }
+    if (ok && (ok = consumer_wait(o_ready, (n - 1) & 1, w))) {
+      tc_fence_after();
+      const float inv_l = p.o_scale / l;
+      const bool valid = qrow < p.N;
+      const size_t row_idx = (size_t)(U.b * p.Hq + U.h) * p.N + qrow;
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row_idx * D);
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tO + cc * 32, r);
+        tmem_ld_wait(r);
+        if (valid) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 pk4;
+            const int i = v4 * 8;
+            pk4.x = pack_bf16x2(__uint_as_float(r[i + 0]) * inv_l, __uint_as_float(r[i + 1]) * inv_l);
+            pk4.y = pack_bf16x2(__uint_as_float(r[i + 2]) * inv_l, __uint_as_float(r[i + 3]) * inv_l);
+            pk4.z = pack_bf16x2(__uint_as_float(r[i + 4]) * inv_l, __uint_as_float(r[i + 5]) * inv_l);
+            pk4.w = pack_bf16x2(__uint_as_float(r[i + 6]) * inv_l, __uint_as_float(r[i + 7]) * inv_l);
+            dst[cc * 4 + v4] = pk4;
+          }
+        }
+      }
+      if (valid) p.lse[row_idx] = (m_ref * c + log2f(l)) * 0.6931471805599453f;
+    }
+  } else {
+    regs_dec<kRegsControl, kRegsLaunch>();  // warps 2-3 and 8-11 have no role here
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 template <int D, int KIND>
 cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                          cudaStream_t stream) {
@@ -603,15 +922,26 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   return cudaGetLastError();
 }
 
+cudaError_t launch_fwd256(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                          cudaStream_t stream) {
+  static_assert(Fwd256Cfg::kSmemBytes <= 232448, "shared memory budget");
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = ensure_smem_limit(fwd256_kernel, Fwd256Cfg::kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
+  const long long units = (long long)p.B * p.Hq * p.n_qblk;
+  fwd256_kernel<<<(unsigned)units, kFwdThreads, Fwd256Cfg::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int d, cudaStream_t s) {
-  if (d == 256) return launch_fwd_d<256, kKindBf16>(tq, tk, tv, p, s);
+  if (d == 256) return launch_fwd256(tq, tk, tv, p, s);
   return d == 128 ? launch_fwd_d<128, kKindBf16>(tq, tk, tv, p, s) : launch_fwd_d<64, kKindBf16>(tq, tk, tv, p, s);
 }
 
-int fwd_tiles_per_cta(int d) { return d == 256 ? FwdCfg<256, false>::kTiles : 2; }
+int fwd_tiles_per_cta(int d) { return d == 256 ? 1 : 2; }
 
 cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, cudaStream_t s) {
