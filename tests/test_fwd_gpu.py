@@ -98,18 +98,22 @@ def test_bf16_fwd_d256(cuda_device, shape, causal):
     check_full(w, cuda_device)
 
 
-def test_bf16_fwd_spiked_rows_force_rescales(cuda_device):
+@pytest.mark.parametrize("d", [64, 256])
+def test_bf16_fwd_spiked_rows_force_rescales(cuda_device, d):
     """Query rows x20 make late key tiles raise the running max far above the
     lazy-rescale threshold."""
-    w = synth.small(1, 4, 4, 1024, 64, True, seed=99, spike_frac=0.05, spike_mul=20.0)
+    w = synth.small(1, 4, 4, 1024, d, True, seed=99, spike_frac=0.05, spike_mul=20.0)
     check_full(w, cuda_device)
 
 
-def test_bf16_fwd_increasing_scores_rescale_every_tile(cuda_device):
-    """Keys that grow along the sequence raise every row's max at each new tile."""
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_bf16_fwd_increasing_scores_rescale_every_tile(cuda_device, d):
+    """Keys that grow along the sequence raise every row's max at each new tile
+    (at d = 256 the rescale waits for the previous P V product, which runs beside
+    the softmax)."""
     import torch
     import exact_io_aware_44_b200 as fa
-    N, d = 1024, 128
+    N = 1024
     rng = np.random.default_rng(5)
     q = synth.round_to_bf16(np.abs(rng.standard_normal((1, 1, N, d))).astype(np.float32))
     ramp = np.linspace(0.0, 3.0, N, dtype=np.float32)[:, None]
@@ -242,4 +246,18 @@ def test_progress_record_counts_each_ctas_work(cuda_device):
     fa.bwd(q, k, v, o, lse, do, causal=True)
     # key tiles 0, 1, 2 of the one kv head see 3, 2, 1 query tiles of each of 2 query heads
     assert sorted(fa.get_progress(3)) == [2, 4, 6]
+    assert fa.get_status() == 0
+
+
+def test_progress_record_d256(cuda_device):
+    """d = 256 runs one 128-row query tile per CTA: each CTA issues as many P V
+    products as its tile visits key tiles."""
+    import torch
+    import exact_io_aware_44_b200 as fa
+    w = synth.small(1, 2, 1, 300, 256, True, seed=5)
+    q, k, v = (to_dev(synth.tensor(w, t), torch.bfloat16, cuda_device)
+               for t in (synth.TID_Q, synth.TID_K, synth.TID_V))
+    fa.fwd(q, k, v, causal=True)
+    # 2 heads x 3 query tiles, which visit 1, 2 and 3 key tiles
+    assert sorted(fa.get_progress(6)) == [1, 1, 2, 2, 3, 3]
     assert fa.get_status() == 0
