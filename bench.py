@@ -592,9 +592,10 @@ def run_ours(args, w, world, rank, local):
 def other_configs(args, fa, torch, dev, stream, peak):
     """The remaining workloads the utilisation targets name, timed after the main
     line on the same device: the c4 forward, the c5 forward and backward, the c2
-    (d = 64) forward and backward, and two decode steps (dec, dec8). Same timing as
-    the main line: CUDA events around each launch on the launching stream, after
-    warm-up, no parity work inside. Inputs: c4, c5 and decode are drawn on the device by a
+    (d = 64) forward and backward, two decode steps (dec, dec8), and the d = 256
+    forward (c6). Same timing as the main line: CUDA events around each launch on the
+    launching stream, after warm-up, no parity work inside. Inputs: c4, c5, c6 and decode
+    are drawn on the device by a
     seeded torch generator with the workloads' distributions (iid N(0, 1)), since
     they are larger than L2 and drawing them on the host would dominate the run;
     c2 uses the parity tests' seeded host recipe (with its spiked rows) and, being
@@ -689,7 +690,7 @@ def other_configs(args, fa, torch, dev, stream, peak):
         x = torch.randn((wl.B, heads, wl.N, wl.d), generator=gen, device=dev, dtype=torch.float32)
         return (x * wl.std).to(torch.bfloat16)
 
-    for name in ("c4", "c5"):
+    for name in ("c4", "c5", "c6"):
         wl = synth.WORKLOADS[name]
         ts = [dev_randn(wl, tid, wl.Hq if tid in (synth.TID_Q, synth.TID_DO) else wl.Hkv)
               for tid in ((synth.TID_Q, synth.TID_K, synth.TID_V) + ((synth.TID_DO,) if wl.backward else ()))]
