@@ -41,6 +41,10 @@ if ROOT not in sys.path:
 METRIC = "attention fwd/bwd TFLOP/s on 1 B200 and % of dense BF16 tensor peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+# fp32 on the CUDA cores (the fp32 forward's roofline): 148 SMs x 128 fp32 lanes x 2 FLOP
+# per FMA x the 1965 MHz maximum SM clock, a nominal figure (no fp32 peak is measured)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+L2_BYTES = 126 << 20
 
 # DRAM bytes (read + write) per launch of the dominant kernel from one ncu
 # capture, with the hash of the kernel source it was taken on. A changed
@@ -313,9 +317,10 @@ def run_ours(args, w, world, rank, local):
     peaks, peak_src = load_peaks()
     fp8 = w.dtype in ("e4m3", "e5m2")
     e5m2 = w.dtype == "e5m2"
+    f32 = w.dtype == "f32"  # the fp32 forward on the CUDA cores
     # dense FP8 peak = measured bf16 x the nominal 2x (4.5 vs 2.25 PFLOP/s dense)
     peak_mul = 2.0 if fp8 else 1.0
-    peak = float(peaks["bf16_tflops"]) * peak_mul
+    peak = FP32_ALU_TFLOPS if f32 else float(peaks["bf16_tflops"]) * peak_mul
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
 
@@ -326,7 +331,8 @@ def run_ours(args, w, world, rank, local):
     # inputs: generated on the host (seeded), kept pinned for the e2e leg
     host = {}
     tids = (("q", synth.TID_Q), ("k", synth.TID_K), ("v", synth.TID_V)) + ((("do", synth.TID_DO),) if w.backward else ())
-    in_dtype = (torch.float8_e5m2 if e5m2 else torch.float8_e4m3fn) if fp8 else torch.bfloat16
+    in_dtype = ((torch.float8_e5m2 if e5m2 else torch.float8_e4m3fn) if fp8
+                else torch.float32 if f32 else torch.bfloat16)
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
     share = 1.0
     if args.shard == "heads":
@@ -342,8 +348,14 @@ def run_ours(args, w, world, rank, local):
     d_in = {n: t.to(dev) for n, t in host.items()}
     if args.shard == "heads":
         B, Hq, Hkv = 1, q1 - q0, k1 - k0
-    o = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=dev)
+    o = torch.empty((B, Hq, N, d), dtype=torch.float32 if f32 else torch.bfloat16, device=dev)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    # Inputs and outputs smaller than L2 would stay cached from one step to the next: then a
+    # buffer larger than L2 is overwritten before every timed step, outside the step's events.
+    step_bytes = sum(t.numel() * t.element_size() for t in d_in.values()) + o.numel() * o.element_size()
+    if w.backward:
+        step_bytes += o.numel() * o.element_size() * 2 + (B * Hkv * N * d * 2) * 2
+    l2_flush = torch.empty(4 * L2_BYTES, dtype=torch.uint8, device=dev) if step_bytes < 2 * L2_BYTES else None
     if w.backward:
         dq = torch.empty_like(o)
         dk = torch.empty((B, Hkv, N, d), dtype=torch.bfloat16, device=dev)
@@ -360,9 +372,9 @@ def run_ours(args, w, world, rank, local):
                                 w.causal, w.scale, sp, e5m2=e5m2)
         else:
             rc = fa.fwd_raw(P(d_in["q"]), P(d_in["k"]), P(d_in["v"]), P(o), P(lse), B, Hq, Hkv, N, d, w.causal,
-                            w.scale, sp)
+                            w.scale, sp, f32=f32)
         if rc:
-            raise fa.FAError(rc, "fa_fwd_fp8" if fp8 else "fa_fwd")
+            raise fa.FAError(rc, "fa_fwd_fp8" if fp8 else "fa_fwd_f32" if f32 else "fa_fwd")
         if not w.backward:
             if events is not None:
                 for e in events[1:]:
@@ -394,6 +406,8 @@ def run_ours(args, w, world, rank, local):
         clocks.mark(True)
         t_start.record(stream)
         for i in range(K):
+            if l2_flush is not None:
+                l2_flush.fill_(i & 0xFF)
             step(evs[i])
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -403,6 +417,8 @@ def run_ours(args, w, world, rank, local):
     if st:
         raise fa.FAError(st, "timed region")
     ms_total = t_start.elapsed_time(t_end)
+    if l2_flush is not None:  # the steps' own spans, without the overwrites between them
+        ms_total = sum(e[0].elapsed_time(e[4]) for e in evs)
     ms_step = reduce_max(ms_total / K)
     # events: 0 fwd start, 1 bwd pre start (= fwd end), 2 main start, 3 convert start, 4 bwd end
     per_kernel = {name: [e[i].elapsed_time(e[i + 1]) for e in evs]
@@ -430,11 +446,12 @@ def run_ours(args, w, world, rank, local):
     rec = NCU_TRAFFIC.get((dominant, w.name))
     if rec and rec.get("csrc_sha") == kernel_source_hash(src_name):
         traffic = rec["bytes_per_launch"]
-    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": UNIT,
+    roofline = {"bound": "alu" if f32 else "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": UNIT,
                 "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": dominant,
-                "peak_source": (f"{peak_src} dense bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
-                                if peak_src == "measured" else "fallback 1.59 PFLOP/s")
-                + (" x 2, the nominal dense fp8:bf16 ratio" if fp8 else ""),
+                "peak_source": ("nominal fp32 FMA rate: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz" if f32 else
+                                (f"{peak_src} dense bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
+                                 if peak_src == "measured" else "fallback 1.59 PFLOP/s")
+                                + (" x 2, the nominal dense fp8:bf16 ratio" if fp8 else "")),
                 "frac_of_sustained": round(achieved / (float(peaks.get("bf16_tflops_sustained", peak)) * peak_mul),
                                            4),
                 # achieved/frac above use the mean launch time over the timed steps; these the median
@@ -463,7 +480,7 @@ def run_ours(args, w, world, rank, local):
                                     B, Hq, Hkv, N, d, w.causal, w.scale, sptr, e5m2=e5m2)
             else:
                 rc = fa.fwd_raw(P(ins["q"]), P(ins["k"]), P(ins["v"]), P(outs["o"]), P(outs["lse"]), B, Hq, Hkv, N,
-                                d, w.causal, w.scale, sptr)
+                                d, w.causal, w.scale, sptr, f32=f32)
             if rc:
                 raise fa.FAError(rc, "fa_fwd")
             if w.backward:
@@ -554,9 +571,13 @@ def run_ours(args, w, world, rank, local):
                                f"{'causal' if w.causal else 'non-causal'} {w.dtype} "
                                f"{'fwd+bwd' if w.backward else 'fwd'}",
                    "B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "causal": w.causal,
-                   "l2": "inputs larger than L2 ("
-                         + ("Q, K, V, O, dO are" if w.backward else "Q, K, V are")
-                         + f" {B * Hq * N * d * (1 if fp8 else 2) / 1e6:.0f} MB each; L2 is 126 MB)",
+                   "l2": ("inputs larger than L2 ("
+                          + ("Q, K, V, O, dO are" if w.backward else "Q, K, V are")
+                          + f" {B * Hq * N * d * (1 if fp8 else 4 if f32 else 2) / 1e6:.0f} MB each; L2 is 126 MB)"
+                          if l2_flush is None else
+                          f"L2 flushed: a {4 * L2_BYTES >> 20} MB buffer is overwritten before every timed step "
+                          f"(the step's tensors, {step_bytes / 1e6:.1f} MB, would fit in the 126 MB L2); the step "
+                          "time sums the steps' own event spans, without the overwrites"),
                    "parallelism": f"head shards x{world}" if args.shard == "heads" else f"replicas x{world}"},
         "pct_of_peak": round(100 * value / world / peak, 2),
         "fwd_tflops": round(kernels["fwd"]["tflops"], 1),
@@ -572,9 +593,9 @@ def run_ours(args, w, world, rank, local):
         # this path moves only the O(N) tensors (algorithmic bytes; ncu-measured DRAM
         # bytes of the dominant kernel in `roofline.traffic`).
         "traffic_model": {"standard_attention_bytes": 8 * B * Hq * N * N,
-                          # Q, K, V read (input dtype), O written (bf16), LSE written (fp32)
-                          "fwd_algorithmic_bytes": (B * Hq + 2 * B * Hkv) * N * d * (1 if fp8 else 2)
-                          + B * Hq * N * d * 2 + B * Hq * N * 4,
+                          # Q, K, V read (input dtype), O written (bf16; fp32 for fp32 inputs), LSE written (fp32)
+                          "fwd_algorithmic_bytes": (B * Hq + 2 * B * Hkv) * N * d * (1 if fp8 else 4 if f32 else 2)
+                          + B * Hq * N * d * (4 if f32 else 2) + B * Hq * N * 4,
                           "bwd_workspace_bytes": fa.workspace_bytes(B, Hq, Hkv, N, d) if w.backward else 0,
                           "note": "the workspace is linear in N (D and the fp32 dQ accumulator); "
                                   "no N x N buffer exists"},
@@ -922,7 +943,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c3",
-                    help="c2, c3, c3n, c5, c6b (bf16 fwd+bwd), c4, c6 (bf16 fwd), f3, f4 (E4M3 fwd), f5 (E5M2 fwd), dec, dec4, dec8 (decode)")
+                    help="c2, c3, c3n, c5, c6b (bf16 fwd+bwd), c4, c6 (bf16 fwd), c1 (fp32 fwd), f3, f4 (E4M3 fwd), "
+                         "f5 (E5M2 fwd), dec, dec4, dec8 (decode)")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N>1: every rank runs the whole workload (weak scaling) or its slice of the heads (strong)")
     ap.add_argument("--e2e-steps", type=int, default=20)

@@ -21,6 +21,38 @@ namespace {
 constexpr int kBr = 32;
 constexpr int kBc = 32;
 constexpr int kF32Threads = 128;
+constexpr int kLoadBatch = 8;  // float4 loads a thread has in flight at once
+
+// Copy `rows` rows of d floats (row-major, 16-byte aligned rows: d % 4 == 0) from global
+// memory at src + r0 * d into shared memory with row pitch `pitch`; rows past n read as
+// zero. Each thread issues kLoadBatch 16-byte loads before it stores any of them, so the
+// loads' latencies overlap instead of following one another.
+__device__ __forceinline__ void load_rows_f32(float* dst, int pitch, const float* src, int r0, int rows, int n,
+                                              int d) {
+  const int n4 = rows * d / 4;
+  for (int e0 = 0; e0 < n4; e0 += kF32Threads * kLoadBatch) {
+    float4 v[kLoadBatch];
+#pragma unroll
+    for (int u = 0; u < kLoadBatch; ++u) {
+      const int e = e0 + u * kF32Threads + (int)threadIdx.x;
+      const int rr = (e * 4) / d, cc = (e * 4) % d;
+      v[u] = (e < n4 && r0 + rr < n) ? *reinterpret_cast<const float4*>(src + (size_t)(r0 + rr) * d + cc)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kLoadBatch; ++u) {
+      const int e = e0 + u * kF32Threads + (int)threadIdx.x;
+      if (e < n4) {
+        const int rr = (e * 4) / d, cc = (e * 4) % d;
+        float* t = dst + rr * pitch + cc;
+        t[0] = v[u].x;
+        t[1] = v[u].y;
+        t[2] = v[u].z;
+        t[3] = v[u].w;
+      }
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kF32Threads) fwd_f32_kernel(const FwdF32Params p) {
   extern __shared__ float sm[];
@@ -47,10 +79,7 @@ __global__ void __launch_bounds__(kF32Threads) fwd_f32_kernel(const FwdF32Params
   const float* kg = p.k + ((size_t)kvh * p.N) * d;
   const float* vg = p.v + ((size_t)kvh * p.N) * d;
 
-  for (int e = tid; e < kBr * d; e += kF32Threads) {
-    const int rr = e / d, cc = e % d;
-    sQ[rr * ldq + cc] = (q0 + rr < p.N) ? qg[(size_t)(q0 + rr) * d + cc] : 0.f;
-  }
+  load_rows_f32(sQ, ldq, qg, q0, kBr, p.N, d);
 
   const float c = p.scale_log2;
   float m = -INFINITY, l = 0.f;
@@ -64,12 +93,8 @@ __global__ void __launch_bounds__(kF32Threads) fwd_f32_kernel(const FwdF32Params
   for (int j = 0; j < n_kv; ++j) {
     const int k0 = j * kBc;
     __syncthreads();  // previous tile's K, V and P are no longer read
-    for (int e = tid; e < kBc * d; e += kF32Threads) {
-      const int rr = e / d, cc = e % d;
-      const bool in = k0 + rr < p.N;
-      sK[rr * ldq + cc] = in ? kg[(size_t)(k0 + rr) * d + cc] : 0.f;
-      sV[rr * d + cc] = in ? vg[(size_t)(k0 + rr) * d + cc] : 0.f;
-    }
+    load_rows_f32(sK, ldq, kg, k0, kBc, p.N, d);
+    load_rows_f32(sV, d, vg, k0, kBc, p.N, d);
     __syncthreads();
 
     float s[8];
