@@ -57,7 +57,7 @@ NCU_TRAFFIC = {
     # profiles/fwd_bf16_d128_B2H32N8192_causal.md, profiles/fwd_bf16_d256_B2H16N8192_causal.md
     ("fwd", "c3"): {"bytes_per_launch": 403438592 + 117224192, "csrc_sha": "85dafde070e56230"},
     ("fwd", "c4"): {"bytes_per_launch": 809460992 + 260929024, "csrc_sha": "85dafde070e56230"},
-    ("fwd", "c6"): {"bytes_per_launch": 403382784 + 117740544, "csrc_sha": "5c1e596934a411c6"},
+    ("fwd", "c6"): {"bytes_per_launch": 403382784 + 117740544, "csrc_sha": "cf21b29ae75def4a"},
     # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md, profiles/decode_wide_B16Hq64Hkv8Nq8_Nk32768_d128.md
     ("decode_split", "dec"): {"bytes_per_launch": 2148459264 + 3497728, "csrc_sha": "91306dfb6f4e6182"},
     ("decode_split", "dec4"): {"bytes_per_launch": 1074816512 + 4360448, "csrc_sha": "91306dfb6f4e6182"},

@@ -562,8 +562,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 // The O tile takes 256 TMEM columns, which leaves room for two score buffers, so the
 // scores of key tile j+1 are computed while the softmax works on tile j, and the
 // chain P(j) -> P V(j) -> S(j+1) -> softmax(j+1) of the one-buffer design leaves the
-// critical path: the softmax runs back to back while the tensor core does P V(j-1)
-// and S(j+1) beside it.
+// critical path: the tensor core does P V(j-1) and S(j+1) while the softmax works. What
+// bounds it then is the tensor core itself: an S product reads both operands from shared
+// memory (8 KB per 64-cycle MMA, the SM's whole shared-memory bandwidth) while the K/V
+// loads write into it, so it runs at about 60 % of the MMA rate.
 //   TMEM: S buffers [0,128) and [128,256) (key tile parity), O [256,512).
 //   warp 0      TMA producer: Q (64 KB), then K and V in 32 KB halves (128 of the
 //               256 columns) through a ring of 5 stages, in the order the MMAs use
