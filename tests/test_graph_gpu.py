@@ -20,15 +20,17 @@ from tests.parity import BWD_REL_FRO, assert_fwd_ok, fwd_errors, rel_fro, to_dev
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [True, False])
-def test_fwd_bwd_decode_captured_and_replayed(cuda_device, causal):
+def test_fwd_bwd_decode_captured_and_replayed(cuda_device, causal, d):
     import torch
 
     import exact_io_aware_44_b200 as fa
-    w = synth.small(1, 8, 2, 700, 128, causal, seed=9100 + causal)
+    w = synth.small(1, 8, 2, 700, d, causal, seed=9100 + causal + d)
     arrs = [synth.tensor(w, t) for t in (synth.TID_Q, synth.TID_K, synth.TID_V, synth.TID_DO)]
     q, k, v, do = (to_dev(x, torch.bfloat16, cuda_device) for x in arrs)
-    dw = synth.DecodeWorkload("graph_dec", 2, 16, 2, 4, 1500, 128, causal, 9200 + causal)  # 32 rows a group
+    dd = 64 if d == 64 else 128  # decode runs d = 64 and 128
+    dw = synth.DecodeWorkload("graph_dec", 2, 16, 2, 4, 1500, dd, causal, 9200 + causal)  # 32 rows a group
     dq_np, dk_np, dv_np = synth.decode_inputs(dw)
     qd, kd, vd = (to_dev(x, torch.bfloat16, cuda_device) for x in (dq_np, dk_np, dv_np))
 
@@ -39,7 +41,7 @@ def test_fwd_bwd_decode_captured_and_replayed(cuda_device, causal):
     ws = torch.empty(fa.workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d), dtype=torch.uint8, device=cuda_device)
     od = torch.empty_like(qd)
     lsed = torch.empty(qd.shape[:3], dtype=torch.float32, device=cuda_device)
-    wsd = torch.empty(fa.decode_workspace_bytes(dw.B, dw.Hq, dw.Hkv, dw.Nq, dw.Nk, 128), dtype=torch.uint8,
+    wsd = torch.empty(fa.decode_workspace_bytes(dw.B, dw.Hq, dw.Hkv, dw.Nq, dw.Nk, dd), dtype=torch.uint8,
                       device=cuda_device)
 
     def step(stream=None):
