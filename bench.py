@@ -59,9 +59,9 @@ NCU_TRAFFIC = {
     ("fwd", "c4"): {"bytes_per_launch": 809460992 + 260929024, "csrc_sha": "85dafde070e56230"},
     ("fwd", "c6"): {"bytes_per_launch": 403382784 + 117740544, "csrc_sha": "cf21b29ae75def4a"},
     # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md, profiles/decode_wide_B16Hq64Hkv8Nq8_Nk32768_d128.md
-    ("decode_split", "dec"): {"bytes_per_launch": 2148459264 + 3497728, "csrc_sha": "91306dfb6f4e6182"},
-    ("decode_split", "dec4"): {"bytes_per_launch": 1074816512 + 4360448, "csrc_sha": "91306dfb6f4e6182"},
-    ("decode_split", "dec8"): {"bytes_per_launch": 2153745920 + 7677696, "csrc_sha": "91306dfb6f4e6182"},
+    ("decode_split", "dec"): {"bytes_per_launch": 2148207360 + 3522816, "csrc_sha": "ca5156f49b56471f"},
+    ("decode_split", "dec4"): {"bytes_per_launch": 1074816000 + 4171776, "csrc_sha": "ca5156f49b56471f"},
+    ("decode_split", "dec8"): {"bytes_per_launch": 2153727488 + 7891456, "csrc_sha": "ca5156f49b56471f"},
 }
 
 

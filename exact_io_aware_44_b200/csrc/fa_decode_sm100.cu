@@ -526,7 +526,9 @@ struct DecWideCfg {
   static constexpr int kColS = 0, kColO = 256;
 };
 
-template <int D>
+// DUP: the block's rows 64-127 repeat rows 0-63 (p.dup), lanes 64-127 taking keys 64-127 of
+// every chunk; a template parameter so that the other blocks' code stays as it was
+template <int D, bool DUP>
 __global__ void __launch_bounds__(DecWideCfg<D>::kThreads, 1)
     decode_split_wide_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                              const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
@@ -636,6 +638,17 @@ __global__ void __launch_bounds__(DecWideCfg<D>::kThreads, 1)
     auto issue_s = [&](int c, const ChunkPos& ps) -> bool {
       if (c == 0 || ps.cig == 0) {
         if (!warp_wait_spin(q_full, ps.seg & 1, w)) return false;
+        if constexpr (DUP) {
+          // rows 64-127 of every 64-column block := rows 0-63 (8 KB each; a row's 128-byte
+          // swizzle depends on the row mod 8, which the copy keeps), for the tensor core
+          constexpr int kPer = C::kRegion / 2 / 16;  // 16-byte pieces of half a block
+          for (int i = lane; i < C::kRegions * kPer; i += 32) {
+            uint8_t* src = smem + C::kOffQ + (i / kPer) * C::kRegion + (i % kPer) * 16;
+            *reinterpret_cast<uint4*>(src + C::kRegion / 2) = *reinterpret_cast<const uint4*>(src);
+          }
+          fence_async_smem();
+          __syncwarp();
+        }
       }
       if (!warp_wait_spin(&kv_full[c % S], (c / S) & 1, w)) return false;
       tc_fence_after();
@@ -720,7 +733,8 @@ __global__ void __launch_bounds__(DecWideCfg<D>::kThreads, 1)
       const bool seg_first = c == 0 || pos.cig == 0;
       const bool seg_last = c == n - 1 || pos.cig == nch - 1;
       if (seg_first) {
-        const int j = (pos.G % p.n_rb) * C::kBlockRows + r;  // row of the group: query j mod Nq of its head
+        // row of the group: query j mod Nq of its head (with dup, lanes r and r + 64 hold row r)
+        const int j = DUP ? (r & 63) : (pos.G % p.n_rb) * C::kBlockRows + r;
         m_ref = -INFINITY;
         l = 0.f;
         lim = j >= p.rows ? -1 : (p.causal ? p.Nk - p.Nq + j % p.Nq : p.Nk - 1);
@@ -732,7 +746,11 @@ __global__ void __launch_bounds__(DecWideCfg<D>::kThreads, 1)
       constexpr int kHalf = kDecChunk / 2;
       float x[kHalf];
       float mx = -INFINITY;
-      if (!dead) {
+      // with dup, lanes 0-63 take keys [0, 64) of the chunk and lanes 64-127 keys [64, 128);
+      // the warpgroup of the other half only stores zeros for P (and still writes its
+      // columns of O at the end)
+      const bool keys_off = DUP && h != (quarter >> 1);
+      if (!dead && !keys_off) {
 #pragma unroll
         for (int cc = 0; cc < kHalf / 32; ++cc) {
           uint32_t rr[32];
@@ -742,7 +760,9 @@ __global__ void __launch_bounds__(DecWideCfg<D>::kThreads, 1)
           for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(rr[i]) * c2;
         }
         const int k0 = pos.cig * kDecChunk + h * kHalf;
-        if (k0 + kHalf - 1 > all_vis || lim < 0) {  // the causal edge, keys past Nk, rows past the end
+        // the causal edge and keys past Nk; rows past the group's end (lim < 0) are left
+        // unmasked: their results are never written, and masking them cost a loop per chunk
+        if (k0 + kHalf - 1 > all_vis) {
 #pragma unroll
           for (int i = 0; i < kHalf; ++i)
             if (k0 + i > lim) x[i] = -INFINITY;
@@ -776,7 +796,7 @@ __global__ void __launch_bounds__(DecWideCfg<D>::kThreads, 1)
       }
       const float mc = m_ref == -INFINITY ? 0.f : m_ref;
       uint32_t pk[kHalf / 2];
-      if (!dead) {
+      if (!dead && !keys_off) {
         uint64_t rs2 = f2_pack(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < kHalf; i += 2) {
@@ -886,9 +906,9 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock) decode_merge_kernel(c
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-#pragma unroll 4
-  for (int i = i0; i <= i1; ++i) {
-    const size_t slot_row = (size_t)(G + i) * p.slot_rows + sq;
+  // one partial row (o_part, lse_part at slot_row) into the running merge (the same steps
+  // as the loop below, which the single-partial case keeps as it was measured)
+  auto take = [&](size_t slot_row) {
     const float ls = p.lse_part[slot_row];
     float o[kPer];
     const float* src = p.o_part + slot_row * D + lane * kPer;
@@ -899,7 +919,7 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock) decode_merge_kernel(c
       const float2 v = *reinterpret_cast<const float2*>(src);
       o[0] = v.x, o[1] = v.y;
     }
-    if (ls == -INFINITY) continue;  // no visible key in this segment
+    if (ls == -INFINITY) return;  // no visible key in this segment
     const float m_new = fmaxf(m, ls);
     const float a = __expf(m - m_new);  // 0 while m is still -inf
     const float wgt = __expf(ls - m_new);
@@ -907,6 +927,38 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock) decode_merge_kernel(c
 #pragma unroll
     for (int e = 0; e < kPer; ++e) acc[e] = acc[e] * a + wgt * o[e];
     m = m_new;
+  };
+  if (p.dup) {
+    // each CTA's slot holds two partial rows of the query row, sq and sq + 64 (one per half
+    // of every key chunk)
+#pragma unroll 2
+    for (int i = i0; i <= i1; ++i) {
+      take((size_t)(G + i) * p.slot_rows + sq);
+      take((size_t)(G + i) * p.slot_rows + sq + 64);
+    }
+  } else {
+#pragma unroll 4
+    for (int i = i0; i <= i1; ++i) {
+      const size_t slot_row = (size_t)(G + i) * p.slot_rows + sq;
+      const float ls = p.lse_part[slot_row];
+      float o[kPer];
+      const float* src = p.o_part + slot_row * D + lane * kPer;
+      if constexpr (kPer == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src);
+        o[0] = v.x, o[1] = v.y, o[2] = v.z, o[3] = v.w;
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(src);
+        o[0] = v.x, o[1] = v.y;
+      }
+      if (ls == -INFINITY) continue;  // no visible key in this segment
+      const float m_new = fmaxf(m, ls);
+      const float a = __expf(m - m_new);  // 0 while m is still -inf
+      const float wgt = __expf(ls - m_new);
+      wsum = wsum * a + wgt;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] = acc[e] * a + wgt * o[e];
+      m = m_new;
+    }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   uint32_t packed[kPer / 2];
@@ -938,14 +990,14 @@ cudaError_t launch_decode_r(const CUtensorMap& tq, const CUtensorMap& tk, const 
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool DUP>
 cudaError_t launch_decode_wide(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                const DecodeParams& p, cudaStream_t s) {
   using C = DecWideCfg<D>;
   static std::atomic<uint64_t> configured{0};
-  cudaError_t e = ensure_smem_limit(decode_split_wide_kernel<D>, C::kSmemBytes, configured);
+  cudaError_t e = ensure_smem_limit(decode_split_wide_kernel<D, DUP>, C::kSmemBytes, configured);
   if (e != cudaSuccess) return e;
-  decode_split_wide_kernel<D><<<(unsigned)p.n_ctas, C::kThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
+  decode_split_wide_kernel<D, DUP><<<(unsigned)p.n_ctas, C::kThreads, C::kSmemBytes, s>>>(tq, tk, tv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<D><<<(unsigned)((p.rows_total + kMergeRowsPerBlock - 1) / kMergeRowsPerBlock),
@@ -963,11 +1015,12 @@ int decode_rows_per_cta(int rows, int d) {
 
 cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           cudaStream_t s) {
-  if (p.d == 64) return launch_decode_wide<64>(tq, tk, tv, p, s);
+  if (p.d == 64)
+    return p.dup ? launch_decode_wide<64, true>(tq, tk, tv, p, s) : launch_decode_wide<64, false>(tq, tk, tv, p, s);
   switch (decode_rows_per_cta(p.rows, p.d)) {
     case 16: return launch_decode_r<16>(tq, tk, tv, p, s);
     case 32: return launch_decode_r<32>(tq, tk, tv, p, s);
-    default: return launch_decode_wide<128>(tq, tk, tv, p, s);
+    default: return launch_decode_wide<128, false>(tq, tk, tv, p, s);
   }
 }
 

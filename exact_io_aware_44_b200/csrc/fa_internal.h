@@ -65,6 +65,9 @@ struct DecodeParams {
   int rows;                        // query rows of a GQA group: (Hq / Hkv) * Nq
   int n_rb;                        // row blocks per group (units of the chunk sequence)
   int slot_rows;                   // query rows of a workspace slot (of a row block)
+  int dup;                         // d = 64, at most 64 rows a group (128-row-block kernel): rows r and
+                                   // r + 64 of the block are query row r, lanes 64-127 taking keys
+                                   // 64-127 of every chunk; both write a partial (slot rows r, r + 64)
   int n_chunks;                    // 128-key chunks per row block
   int n_ctas;                      // split-kernel CTAs (equal slices of all row blocks' chunks)
   long long total_chunks;          // B * Hkv * n_rb * n_chunks

@@ -125,7 +125,9 @@ int fa_fwd_e5m2(const void* q, const void* k, const void* v, float descale_q, fl
  * row blocks, each a unit of its own. The split kernel cuts all units' 128-key
  * chunks, laid end to end, into n_ctas equal slices; each piece of a slice inside
  * one unit has a slot holding a float32 partial output [slot_rows, d] and partial
- * LSE [slot_rows], where slot_rows = rows for n_rb = 1 and 128 otherwise; there
+ * LSE [slot_rows], where slot_rows = rows for n_rb = 1 and 128 otherwise, and 128
+ * at d = 64 with rows <= 64 (two partial rows per query row, one per half of
+ * every 128-key chunk); there
  * are units + n_ctas - 1 slots, units = B*Hkv*n_rb. The workspace holds all slots'
  * outputs (padded to a multiple of 256 bytes), then all their LSEs. n_ctas is 148
  * for num_splits <= 0 (a fixed rule of the sizes, so no device is needed here),

@@ -100,15 +100,17 @@ def test_decode_rejects_bad_arguments_on_host():
     assert _dec(ws=0) == -1
 
 
-def _decode_split(B, Hq, Hkv, Nq, Nk, splits):
+def _decode_split(B, Hq, Hkv, Nq, Nk, splits, d=128):
     """The work split restated: a group of up to 32 query rows is one unit, a larger
     one is ceil(rows / 128) row blocks of 128; all units' 128-key chunks end to end,
     cut into n_ctas equal slices (one per SM of a 148-SM part, or units * num_splits;
     never more than the chunks); one workspace slot per (unit, CTA) pair that can
-    meet, i.e. units + n_ctas - 1, each of slot_rows rows."""
+    meet, i.e. units + n_ctas - 1, each of slot_rows rows. At d = 64 a group of at most
+    64 rows keeps two partial rows per query row (one per half of every key chunk), in
+    slots of 128 rows."""
     rows = Hq // Hkv * Nq
     n_rb = 1 if rows <= 32 else -(-rows // 128)
-    slot_rows = rows if n_rb == 1 else 128
+    slot_rows = 128 if (d == 64 and rows <= 64) else rows if n_rb == 1 else 128
     n_chunks = -(-Nk // 128)
     units = B * Hkv * n_rb
     n_ctas = min(units * splits if splits > 0 else 148, units * n_chunks)
@@ -129,10 +131,14 @@ def test_decode_workspace_and_split_rule():
             pad = lambda x: (x + 255) // 256 * 256
             assert ws == pad(slots * slot_rows * d * 4) + slots * slot_rows * 4, (B, Hq, Hkv, Nq, Nk, splits, ws)
     assert fa.decode_workspace_bytes(1, 8, 1, 1, 1000, 256, 0) == 0
-    # d = 64: the same split rule, d = 64 floats per partial row
-    slots, slot_rows, _ = _decode_split(2, 8, 2, 3, 1000, 0)
+    # d = 64: the same split rule, d = 64 floats per partial row; up to 64 rows a group, two
+    # partial rows per query row
     pad = lambda x: (x + 255) // 256 * 256
-    assert fa.decode_workspace_bytes(2, 8, 2, 3, 1000, 64, 0) == pad(slots * slot_rows * 64 * 4) + slots * slot_rows * 4
+    for (B, Hq, Hkv, Nq) in ((2, 8, 2, 3), (16, 64, 8, 8), (2, 8, 1, 9), (1, 16, 1, 40)):
+        slots, slot_rows, _ = _decode_split(B, Hq, Hkv, Nq, 1000, 0, d=64)
+        assert slot_rows == (128 if Hq // Hkv * Nq <= 64 else Hq // Hkv * Nq if Hq // Hkv * Nq <= 128 else 128)
+        assert fa.decode_workspace_bytes(B, Hq, Hkv, Nq, 1000, 64, 0) == \
+            pad(slots * slot_rows * 64 * 4) + slots * slot_rows * 4, (B, Hq, Hkv, Nq)
 
 
 def test_bwd_rejects_bad_arguments_on_host():
