@@ -62,6 +62,7 @@ NCU_TRAFFIC = {
     ("decode_split", "dec"): {"bytes_per_launch": 2148207360 + 3522816, "csrc_sha": "ca5156f49b56471f"},
     ("decode_split", "dec4"): {"bytes_per_launch": 1074816000 + 4171776, "csrc_sha": "ca5156f49b56471f"},
     ("decode_split", "dec8"): {"bytes_per_launch": 2153727488 + 7891456, "csrc_sha": "ca5156f49b56471f"},
+    ("decode_split", "dec64"): {"bytes_per_launch": 1074019328 + 3989504, "csrc_sha": "ca5156f49b56471f"},
 }
 
 
@@ -613,7 +614,7 @@ def run_ours(args, w, world, rank, local):
 def other_configs(args, fa, torch, dev, stream, peak):
     """The remaining workloads the utilisation targets name, timed after the main
     line on the same device: the c4 forward, the c5 forward and backward, the c2
-    (d = 64) forward and backward, two decode steps (dec, dec8), and the d = 256
+    (d = 64) forward and backward, three decode steps (dec, dec8, dec64), and the d = 256
     forward (c6). Same timing as the main line: CUDA events around each launch on the
     launching stream, after warm-up, no parity work inside. Inputs: c4, c5, c6 and decode
     are drawn on the device by a
@@ -724,8 +725,9 @@ def other_configs(args, fa, torch, dev, stream, peak):
          True)
     del ts
     # decode: one new query per head against a 32768-key cache (dec, 4 query rows a group), and
-    # eight new tokens per sequence of a 64-head model (dec8, 64 query rows a group)
-    for dname in ("dec", "dec8"):
+    # eight new tokens per sequence of a 64-head model (dec8, 64 query rows a group), and the
+    # first at a head dim of 64 (dec64)
+    for dname in ("dec", "dec8", "dec64"):
         dw = synth.DECODE_WORKLOADS[dname]
         gen.manual_seed(dw.seed)
         qd = torch.randn((dw.B, dw.Hq, dw.Nq, dw.d), generator=gen, device=dev).to(torch.bfloat16)
@@ -944,7 +946,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c3",
                     help="c2, c3, c3n, c5, c6b (bf16 fwd+bwd), c4, c6 (bf16 fwd), c1 (fp32 fwd), f3, f4 (E4M3 fwd), "
-                         "f5 (E5M2 fwd), dec, dec4, dec8 (decode)")
+                         "f5 (E5M2 fwd), dec, dec4, dec8, dec64 (decode)")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N>1: every rank runs the whole workload (weak scaling) or its slice of the heads (strong)")
     ap.add_argument("--e2e-steps", type=int, default=20)

@@ -266,6 +266,9 @@ DECODE_WORKLOADS = {
     # 8 new tokens per sequence, 64 query heads over 8 kv heads: 64 query rows a group,
     # the 128-row-block kernel
     "dec8": DecodeWorkload("dec8", 16, 64, 8, 8, 32768, 128, True, 1013),
+    # the step of "dec" with a head dim of 64 (4 query rows a group: the 128-row-block kernel
+    # with the rows duplicated over both lane halves)
+    "dec64": DecodeWorkload("dec64", 16, 32, 8, 1, 32768, 64, True, 1014),
 }
 
 

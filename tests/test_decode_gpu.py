@@ -164,12 +164,12 @@ def test_decode_workspace_reused_with_garbage(cuda_device, shape):
                       f"reused workspace splits={splits}")
 
 
-@pytest.mark.parametrize("name", ["dec", "dec4", "dec8"])
+@pytest.mark.parametrize("name", ["dec", "dec4", "dec8", "dec64"])
 def test_decode_full_size_workload(cuda_device, name):
-    """The benchmark's decode steps (B=16 Hq=32 against 32768 cached keys: Hkv=8 with
-    one new query, Hkv=4 with four), in the launch configuration the benchmark
-    times (automatic splits); every output computed, sampled heads checked
-    against the oracle."""
+    """The benchmark's decode steps (B=16 against 32768 cached keys: Hq=32 Hkv=8 with
+    one new query at d = 128 and at d = 64, Hq=32 Hkv=4 with four, Hq=64 Hkv=8 with
+    eight), in the launch configuration the benchmark times (automatic splits); every
+    output computed, sampled heads checked against the oracle."""
     w = synth.DECODE_WORKLOADS[name]
     q, k, v, o, lse = run_decode(w, cuda_device)
     assert np.isfinite(o).all() and np.isfinite(lse).all()
