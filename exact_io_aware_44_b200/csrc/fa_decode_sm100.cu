@@ -772,7 +772,7 @@ __global__ void __launch_bounds__(DecWideCfg<D>::kThreads, 1)
         for (int i = 4; i < kHalf; i += 8) {
           mq[0] = fmax3(mq[0], x[i], x[i + 1]);
           mq[1] = fmax3(mq[1], x[i + 2], x[i + 3]);
-          mq[2] = fmax3(mq[2], x[i + 4], x[i + 5]);
+          if (i + 4 < kHalf) mq[2] = fmax3(mq[2], x[i + 4], x[i + 5]);  // the last step has 4 left
           if (i + 6 < kHalf) mq[3] = fmax3(mq[3], x[i + 6], x[i + 7]);
         }
         mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);

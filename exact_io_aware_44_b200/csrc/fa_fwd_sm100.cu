@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int i = 4; i < kTileN; i += 8) {
           mq[0] = fmax3(mq[0], s[i], s[i + 1]);
           mq[1] = fmax3(mq[1], s[i + 2], s[i + 3]);
-          mq[2] = fmax3(mq[2], s[i + 4], s[i + 5]);
+          if (i + 4 < kTileN) mq[2] = fmax3(mq[2], s[i + 4], s[i + 5]);  // the last step has 4 left
           if (i + 6 < kTileN) mq[3] = fmax3(mq[3], s[i + 6], s[i + 7]);
         }
         const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
@@ -802,7 +802,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int i = 4; i < kTileN; i += 8) {
         mq[0] = fmax3(mq[0], s[i], s[i + 1]);
         mq[1] = fmax3(mq[1], s[i + 2], s[i + 3]);
-        mq[2] = fmax3(mq[2], s[i + 4], s[i + 5]);
+        if (i + 4 < kTileN) mq[2] = fmax3(mq[2], s[i + 4], s[i + 5]);  // the last step has 4 left
         if (i + 6 < kTileN) mq[3] = fmax3(mq[3], s[i + 6], s[i + 7]);
       }
       const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
