@@ -55,14 +55,14 @@ NCU_TRAFFIC = {
     # profiles/bwd_main_d64_B4H16N2048_causal.md
     ("bwd_main", "c2"): {"bytes_per_launch": 101785600 + 24538112, "csrc_sha": "0db9771b218176f6"},
     # profiles/fwd_bf16_d128_B2H32N8192_causal.md, profiles/fwd_bf16_d256_B2H16N8192_causal.md
-    ("fwd", "c3"): {"bytes_per_launch": 403438592 + 117224192, "csrc_sha": "85dafde070e56230"},
-    ("fwd", "c4"): {"bytes_per_launch": 809460992 + 260929024, "csrc_sha": "85dafde070e56230"},
-    ("fwd", "c6"): {"bytes_per_launch": 403382784 + 117740544, "csrc_sha": "cf21b29ae75def4a"},
+    ("fwd", "c3"): {"bytes_per_launch": 403569664 + 117326848, "csrc_sha": "d22978f98dcad723"},
+    ("fwd", "c4"): {"bytes_per_launch": 809743360 + 260787968, "csrc_sha": "d22978f98dcad723"},
+    ("fwd", "c6"): {"bytes_per_launch": 403493888 + 118081024, "csrc_sha": "b1a823b364771c18"},
     # profiles/decode_B16Hq32Hkv8_Nk32768_d128.md, profiles/decode_wide_B16Hq64Hkv8Nq8_Nk32768_d128.md
-    ("decode_split", "dec"): {"bytes_per_launch": 2148207360 + 3522816, "csrc_sha": "ca5156f49b56471f"},
-    ("decode_split", "dec4"): {"bytes_per_launch": 1074816000 + 4171776, "csrc_sha": "ca5156f49b56471f"},
-    ("decode_split", "dec8"): {"bytes_per_launch": 2153727488 + 7891456, "csrc_sha": "ca5156f49b56471f"},
-    ("decode_split", "dec64"): {"bytes_per_launch": 1074019328 + 3989504, "csrc_sha": "ca5156f49b56471f"},
+    ("decode_split", "dec"): {"bytes_per_launch": 2148206592 + 3491072, "csrc_sha": "d4b94526a7290b64"},
+    ("decode_split", "dec4"): {"bytes_per_launch": 1074812160 + 4385280, "csrc_sha": "d4b94526a7290b64"},
+    ("decode_split", "dec8"): {"bytes_per_launch": 2153774592 + 7643648, "csrc_sha": "d4b94526a7290b64"},
+    ("decode_split", "dec64"): {"bytes_per_launch": 1074049792 + 3947520, "csrc_sha": "d4b94526a7290b64"},
 }
 
 
