@@ -51,9 +51,9 @@ L2_BYTES = 126 << 20
 # source makes the figure stale and the bench reports null.
 NCU_TRAFFIC = {
     # profiles/bwd_main_d128_B2H32N8192_causal.md
-    ("bwd_main", "c3"): {"bytes_per_launch": 810053376 + 491489280, "csrc_sha": "eca1cf4d70f597f7"},
+    ("bwd_main", "c3"): {"bytes_per_launch": 810053376 + 491489280, "csrc_sha": "5f1ce705a7c0333f"},
     # profiles/bwd_main_d64_B4H16N2048_causal.md
-    ("bwd_main", "c2"): {"bytes_per_launch": 101785600 + 24538112, "csrc_sha": "0db9771b218176f6"},
+    ("bwd_main", "c2"): {"bytes_per_launch": 101773056 + 22512384, "csrc_sha": "ca60193791cdd550"},
     # profiles/fwd_bf16_d128_B2H32N8192_causal.md, profiles/fwd_bf16_d256_B2H16N8192_causal.md
     ("fwd", "c3"): {"bytes_per_launch": 403569664 + 117326848, "csrc_sha": "d22978f98dcad723"},
     ("fwd", "c4"): {"bytes_per_launch": 809743360 + 260787968, "csrc_sha": "d22978f98dcad723"},
@@ -70,9 +70,11 @@ NCU_TRAFFIC = {
 # to end marker) plus the shared device helpers. Edits elsewhere in the file (the
 # other head-dim variant, comments) leave the recorded counters valid.
 KERNEL_SOURCES = {
-    "bwd_main": ("fa_bwd_sm100.cu", [("__device__ __forceinline__ void red_add(", "// ----"),
+    "bwd_main": ("fa_bwd_sm100.cu", [("#ifndef FA_BWD_POLY_PAIRS", "// Register split: the launch gives"),
+                                     ("__device__ __forceinline__ void red_add(", "// ----"),
                                      ("struct Bwd128Cfg {", "struct Bwd64Cfg {")]),
-    "bwd_main_d64": ("fa_bwd_sm100.cu", [("struct Bwd64Cfg {", "template <int D>\ncudaError_t launch_preprocess_d(")]),
+    "bwd_main_d64": ("fa_bwd_sm100.cu", [("#ifndef FA_BWD_POLY_PAIRS", "// Register split: the launch gives"),
+                                         ("struct Bwd64Cfg {", "template <int D>\ncudaError_t launch_preprocess_d(")]),
     "fwd": ("fa_fwd_sm100.cu", [("constexpr int kFwdThreads = 384;", "// fwd256_kernel (bf16")]),
     "fwd256": ("fa_fwd_sm100.cu", [("constexpr int kFwdThreads = 384;", "template <int D, bool FP8>\nstruct FwdCfg {"),
                                    ("struct FwdUnit {", "// PERSIST: the grid"),

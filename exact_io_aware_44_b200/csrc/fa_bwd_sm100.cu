@@ -47,6 +47,10 @@ constexpr int kBwdThreads = 512;
 // Of every 8 pairs of P^T values, how many take 2^x by polynomial on the FMA pipe
 // instead of the SFU (128-row kernel).
 constexpr int kBwdPolyPairs = FA_BWD_POLY_PAIRS;
+#ifndef FA_BWD64_POLY_PAIRS
+#define FA_BWD64_POLY_PAIRS 1
+#endif
+constexpr int kBwd64PolyPairs = FA_BWD64_POLY_PAIRS;  // the same, for the d = 64 kernel
 // Register split: the launch gives 128 per thread (512 x 128 = 65536). The
 // control and dQ warpgroups lower to 96 and the two P/dS warpgroups raise to
 // 160: 128 x (96 + 2 x 160 + 96) = 65536.
@@ -945,8 +949,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const ulonglong2 nv = nl4[i / 4];
         float x0, x1;
         f2_unpack(f2_fma(f2_pack(pr[i], pr[i + 1]), c2, (i & 2) ? nv.y : nv.x), x0, x1);
-        pr[i] = ex2(x0);
-        pr[i + 1] = ex2(x1);
+        if (((i / 2) & 7) < kBwd64PolyPairs) {  // part of the exponentials on the FMA pipe
+          ex2_poly2(x0, x1, pr[i], pr[i + 1]);
+        } else {
+          pr[i] = ex2(x0);
+          pr[i + 1] = ex2(x1);
+        }
       }
       if (p.causal && i0 < j0 + kTileN) {  // the diagonal tile only
 #pragma unroll
