@@ -165,6 +165,7 @@ class ClockSampler:
         self._stop = None
         self._thread = None
         self._smi = None
+        self._nv = None  # (module, handle, reasons function, max SM clock) once NVML is up
 
     def _handle(self, nv):
         import torch
@@ -174,16 +175,18 @@ class ClockSampler:
         except Exception:
             return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
-    def _poll(self, nv, h):
-        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-            nv.nvmlDeviceGetCurrentClocksThrottleReasons
-        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+    def _sample(self):
+        """One NVML reading (clock, max clock, power, reasons) appended to the samples."""
+        nv, h, reasons_fn, mx = self._nv
+        try:
+            self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), mx,
+                                 nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(reasons_fn(h))))
+        except Exception:
+            pass
+
+    def _poll(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), mx,
-                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(reasons_fn(h))))
-            except Exception:
-                pass
+            self._sample()
             self._stop.wait(self.interval)
 
     def __enter__(self):
@@ -192,11 +195,15 @@ class ClockSampler:
             import pynvml as nv
             nv.nvmlInit()
             h = self._handle(nv)
+            reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self._nv = (nv, h, reasons_fn, nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
             self._stop = threading.Event()
-            self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self._thread = threading.Thread(target=self._poll, daemon=True)
             self._thread.start()
         except Exception:
             self._thread = None
+            self._nv = None
             self._start_smi()
         time.sleep(0.05)
         return self
@@ -215,7 +222,14 @@ class ClockSampler:
             self._smi = None
 
     def mark(self, start: bool):
-        self.window[0 if start else 1] = time.perf_counter()
+        """Bracket the timed region; with NVML, a reading is taken at each edge too, so that a
+        region shorter than the polling interval still has samples of its own."""
+        if start:
+            self.window[0] = time.perf_counter()
+        if self._nv is not None:
+            self._sample()
+        if not start:
+            self.window[1] = time.perf_counter()
 
     def __exit__(self, *exc):
         time.sleep(0.02)

@@ -113,3 +113,27 @@ def test_reference_arm_prints_one_line_of_the_contract(capsys):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["config"]["workload"].startswith("c1:")
 
+
+
+def test_clock_marks_sample_the_region_edges():
+    """With NVML up, each edge of the timed region takes a reading of its own, so a region
+    shorter than the polling interval is never left without samples (a fake NVML here)."""
+    class FakeNvml:
+        NVML_CLOCK_SM = 0
+
+        @staticmethod
+        def nvmlDeviceGetClockInfo(h, kind):
+            return 1800
+
+        @staticmethod
+        def nvmlDeviceGetPowerUsage(h):
+            return 640_000  # mW
+
+    s = bench.ClockSampler(0)
+    s._nv = (FakeNvml, object(), lambda h: 0x4, 1965)
+    s.mark(True)
+    s.mark(False)
+    summ = s.summary()
+    assert summ["samples"] == 2
+    assert summ["sm_mhz"] == 1800 and summ["sm_max_mhz"] == 1965
+    assert summ["reasons"] == ["sw_power_cap"] and summ["power_w_max"] == 640.0
