@@ -8,7 +8,9 @@
 // exactly once at full bandwidth. A GQA group (one batch entry and kv head: g
 // query heads x Nq queries) of up to 32 rows is the unit that shares K and V
 // (decode_split_kernel<R>); a larger group is cut into 128-row blocks, each a unit
-// (decode_split_wide_kernel, below). A unit's keys form n_chunks chunks of 128.
+// (decode_split_wide_kernel, below; every group at d = 64, where a group of at most
+// 64 rows fills both halves of its block with the same rows, each half taking half of
+// every chunk's keys). A unit's keys form n_chunks chunks of 128.
 // All units' chunks are laid end to end, and CTA i of the persistent grid (one CTA
 // per SM) takes the i-th of n_ctas equal slices of that sequence. A slice may
 // cross unit boundaries: each piece of it that lies in one unit is a segment, with
